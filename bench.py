@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of one hierarchical-local-attention layer on B200.
+
+A step is one pass of the whole layer over one batch of synthetic raster-order
+inputs already resident in HBM: window-first permute of q, k, v (3 launches),
+RoPE of q and k, high-res and low-res (4), block-sparse attention (1),
+unpermute of the output (1).  The metric is useful attention TFLOP/s
+(4 * head_dim FLOPs per visible query-key pair per head) over the step, with
+ms per layer; the attention kernel alone is also timed and set against the
+measured bf16 tensor peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4K] [--impl ug|reference]
+
+N > 1 runs under torchrun, one rank per GPU; every rank runs its own layer on
+its own inputs (independent problems, weak scaling, no data-path collective);
+the time is the max over ranks.  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from block_sparse_local_raster_b200 import workloads  # noqa: E402
+
+METRIC = "useful attn TFLOP/s & ms/layer at 4K/8K token grids; % of B200 bf16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="4K", choices=list(workloads.CONFIGS))
+    ap.add_argument("--impl", default="ug", choices=["ug", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def useful_flops(wl) -> int:
+    from block_sparse_local_raster_b200 import ug
+    pairs = sum(ug.visible_pairs(ug.make_geom(**wl.geom_dict())))
+    return 4 * wl.head_dim * pairs * wl.heads * wl.batch
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(backend: str, world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def reduce_max(x: float, device) -> float:
+    """Max over ranks (identity for a single process)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def aggregate(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed / the slowest rank."""
+    return units_per_rank * world / max_seconds
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        rows = [l.split(", ") for l in open(self.out.name).read().strip().splitlines() if l]
+        os.unlink(self.out.name)
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = max(smax, float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip() == "Active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def attn_traffic_bytes(config: str):
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    if the kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "attention_dram_traffic.json")
+    src = os.path.join(ROOT, "block_sparse_local_raster_b200", "csrc", "ug_attn.cu")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    e = d.get(config)
+    if not e or e.get("source_sha256_16") != h:
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+class OracleArm:
+    """The fp64 CPU oracle on a bounded sample of the workload."""
+
+    def __init__(self, wl, rows_hr: int, rows_lr: int, heads, seed: int = 0):
+        from oracle import hier_local_attn as O
+        self.O = O
+        self.g = O.Geometry.from_dict(wl.geom_dict())
+        x = workloads.make_inputs(wl, seed=seed)
+        self.bits = {k: v.view(torch.int16).numpy().view(np.uint16)
+                     for k, v in x.items() if k != "head_scale"}
+        rng = np.random.default_rng(seed)
+        hr = rng.choice(self.g.N, size=min(rows_hr, self.g.N), replace=False)
+        lr = rng.choice(self.g.L, size=min(rows_lr, self.g.L), replace=False) if self.g.L else []
+        self.rows = np.sort(np.concatenate([hr, self.g.N + np.asarray(lr, dtype=np.int64)]))
+        self.heads = list(heads)
+        # useful FLOPs of the sample: visible keys of each sampled row
+        T = self.g.T
+        off, idx = O.window_neighbours(self.g)
+        perm = O.window_first_index(self.g)
+        vis = 0
+        for r in self.rows:
+            if r < self.g.N:
+                w = perm[r] // T
+                vis += (off[w + 1] - off[w]) * T + self.g.L
+            else:
+                vis += self.g.L
+        self.flops = 4 * self.g.head_dim * vis * len(self.heads) * wl.batch
+
+    def step(self):
+        self.O.layer_forward(self.bits, self.g, self.rows, self.heads)
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    arm = OracleArm(wl, rows_hr=8, rows_lr=2, heads=[0])
+    for _ in range(args.warmup):
+        arm.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        arm.step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = arm.flops / dt / 1e12
+    sample = (f"{len(arm.rows)} query rows ({(arm.rows < arm.g.N).sum()} high-res, "
+              f"{(arm.rows >= arm.g.N).sum()} low-res) x 1 head of the {wl.name} layer per step, "
+              "RoPE of all keys of that head included; fp64 numpy")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_ug(args, wl, world, rank, local):
+    from block_sparse_local_raster_b200 import ug
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl", world)
+    stream = torch.cuda.current_stream(dev)
+
+    plan = ug.Plan(**wl.geom_dict())
+    host = workloads.make_inputs(wl, seed=rank)
+    host.pop("head_scale", None)
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    d = {k: v.to(dev) for k, v in pinned.items()}
+    B, N, H, D = d["q_hr"].shape
+    L = wl.n_lr
+    ws = torch.empty(plan.workspace_bytes(), dtype=torch.uint8, device=dev)
+    o_hr = torch.empty_like(d["q_hr"])
+    o_lr = torch.empty_like(d["q_lr"]) if L else None
+    lse = torch.empty((B, H, N + L), dtype=torch.float32, device=dev)
+    hr_bytes = d["q_hr"].numel() * 2
+    lr_bytes = d["q_lr"].numel() * 2
+    up = lambda n: (n + 255) // 256 * 256
+    # window-first scratch inside the workspace, same split as ug_layer_fwd
+    ws_q = ws[0:hr_bytes].view(torch.bfloat16).view(B, N, H, D)
+    ws_k = ws[up(hr_bytes):up(hr_bytes) + hr_bytes].view(torch.bfloat16).view(B, N, H, D)
+    ws_v = ws[2 * up(hr_bytes):2 * up(hr_bytes) + hr_bytes].view(torch.bfloat16).view(B, N, H, D)
+    ws_o = ws[3 * up(hr_bytes):3 * up(hr_bytes) + hr_bytes].view(torch.bfloat16).view(B, N, H, D)
+    o4 = 4 * up(hr_bytes)
+    ws_ql = ws[o4:o4 + lr_bytes].view(torch.bfloat16).view(B, L, H, D) if L else None
+    ws_kl = ws[o4 + up(lr_bytes):o4 + up(lr_bytes) + lr_bytes].view(torch.bfloat16).view(B, L, H, D) if L else None
+
+    def chk(st, what):
+        if st != ug.UG_OK:
+            raise ug.UgError(st, what)
+
+    def step(ev=None):
+        chk(plan.permute_window_first(d["q_hr"], ws_q), "permute q")
+        chk(plan.permute_window_first(d["k_hr"], ws_k), "permute k")
+        chk(plan.permute_window_first(d["v_hr"], ws_v), "permute v")
+        chk(plan.rope_2d(ws_q, ws_q, ug.UG_HR_WINDOW_FIRST), "rope q")
+        chk(plan.rope_2d(ws_k, ws_k, ug.UG_HR_WINDOW_FIRST), "rope k")
+        if L:
+            chk(plan.rope_2d(d["q_lr"], ws_ql, ug.UG_LR), "rope q_lr")
+            chk(plan.rope_2d(d["k_lr"], ws_kl, ug.UG_LR), "rope k_lr")
+        if ev is not None:
+            ev[0].record(stream)
+        chk(plan.hier_local_attn_fwd(ws_q, ws_k, ws_v, ws_ql, ws_kl, d["v_lr"] if L else None,
+                                     ws_o, o_lr, lse), "attention")
+        if ev is not None:
+            ev[1].record(stream)
+        chk(plan.unpermute(ws_o, o_hr), "unpermute")
+
+    launches_per_step = 3 + 2 + (2 if L else 0) + 1 + 1
+    flops = useful_flops(wl)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = plan.check_error()
+    if st != ug.UG_OK:
+        raise ug.UgError(st, "warm-up")
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(attn_ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    st = plan.check_error()
+    if st != ug.UG_OK:
+        raise ug.UgError(st, "timed steps")
+    sec = t0.elapsed_time(t1) / 1e3 / args.steps
+    attn_sec = sum(a.elapsed_time(b) for a, b in attn_ev) / 1e3 / args.steps
+    sec_max = reduce_max(sec, dev)
+    attn_max = reduce_max(attn_sec, dev)
+
+    # End to end through the public API: pinned host inputs -> device, the
+    # layer (ug_layer_fwd), outputs -> pinned host, every step.
+    out_host = torch.empty_like(o_hr, device="cpu").pin_memory()
+    out_lr_host = torch.empty_like(o_lr, device="cpu").pin_memory() if L else None
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = o_hr.numel() * 2 + (o_lr.numel() * 2 if L else 0)
+
+    def e2e_step():
+        for k in d:
+            d[k].copy_(pinned[k], non_blocking=True)
+        chk(plan.layer_fwd(d["q_hr"], d["k_hr"], d["v_hr"], d["q_lr"] if L else None,
+                           d["k_lr"] if L else None, d["v_lr"] if L else None, o_hr, o_lr, lse,
+                           ws), "ug_layer_fwd")
+        out_host.copy_(o_hr, non_blocking=True)
+        if L:
+            out_lr_host.copy_(o_lr, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_sec = reduce_max(e0.elapsed_time(e1) / 1e3 / args.e2e_steps, dev)
+
+    if rank == 0:
+        pk, pk_src = peaks()
+        achieved = flops / attn_max / 1e12
+        line = {
+            "metric": METRIC,
+            "value": aggregate(flops, world, sec_max) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": sec_max * 1e3,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": wl.name,
+                "batch": wl.batch, "grid": [wl.grid_h, wl.grid_w],
+                "window": [wl.win_h, wl.win_w], "radius": wl.radius,
+                "lowres_grid": [wl.lr_h, wl.lr_w], "rho": wl.rho,
+                "heads": wl.heads, "head_dim": wl.head_dim,
+                "useful_flop_per_layer": flops,
+                "l2": "inputs larger than L2 (each high-res tensor %.0f MB > 126 MB), no flush"
+                      % (hr_bytes / 1e6),
+                "parallelism": f"independent layer per GPU x{world}",
+            },
+            "attn_ms": attn_max * 1e3,
+            "attn_tflops": achieved,
+            "roofline": {
+                "bound": "tensor",
+                "achieved": achieved,
+                "peak": pk["bf16_tflops_sustained"],
+                "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops_sustained"],
+                "traffic": attn_traffic_bytes(wl.name),
+                "peak_source": f"{pk_src} bf16 cuBLAS, sustained (kernel timed inside a long step loop)",
+                "frac_of_burst_peak": achieved / pk["bf16_tflops"],
+            },
+            "e2e": {"value": aggregate(flops, world, e2e_sec) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_sec * 1e3,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            arm = OracleArm(wl, rows_hr=48, rows_lr=8, heads=range(wl.heads))
+            c0 = time.perf_counter()
+            arm.step()
+            cdt = time.perf_counter() - c0
+            line["cpu_baseline"] = {
+                "value": arm.flops / cdt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+                "kind": "oracle",
+                "sample": (f"{len(arm.rows)} query rows x {wl.heads} heads of the {wl.name} "
+                           f"layer (RoPE of every key included), fp64 numpy, {cdt:.1f} s"),
+            }
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_env()
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    wl = workloads.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        return
+    run_ug(args, wl, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

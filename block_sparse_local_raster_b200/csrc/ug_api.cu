@@ -1,0 +1,279 @@
+// The C ABI: argument checks, plan lifetime, the layer sequence.
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "ug_internal.h"
+
+using namespace ug;
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
+  if (!a || !b || na <= 0 || nb <= 0) return false;
+  const char* pa = static_cast<const char*>(a);
+  const char* pb = static_cast<const char*>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+int64_t hr_bytes(const ug_plan* p) {
+  return (int64_t)p->g.batch * p->N * p->g.heads * p->g.head_dim * 2;
+}
+int64_t lr_bytes(const ug_plan* p) {
+  return (int64_t)p->g.batch * p->L * p->g.heads * p->g.head_dim * 2;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ug_geom_validate(const ug_geom* g) { return validate(g); }
+
+int ug_index_map_sizes(const ug_geom* g, int64_t* n_perm, int64_t* n_nbr_off,
+                       int64_t* n_nbr_idx) {
+  int st = validate(g);
+  if (st != UG_OK) return st;
+  const int64_t nwy = g->grid_h / g->win_h, nwx = g->grid_w / g->win_w;
+  std::vector<int32_t> off, idx;
+  build_neighbours(*g, off, idx);
+  if (n_perm) *n_perm = (int64_t)g->grid_h * g->grid_w;
+  if (n_nbr_off) *n_nbr_off = nwy * nwx + 1;
+  if (n_nbr_idx) *n_nbr_idx = (int64_t)idx.size();
+  return UG_OK;
+}
+
+int ug_build_index_maps(const ug_geom* g, int32_t* perm, int32_t* nbr_off, int32_t* nbr_idx) {
+  int st = validate(g);
+  if (st != UG_OK) return st;
+  std::vector<int32_t> p, off, idx;
+  build_perm(*g, p);
+  build_neighbours(*g, off, idx);
+  if (perm) std::memcpy(perm, p.data(), p.size() * sizeof(int32_t));
+  if (nbr_off) std::memcpy(nbr_off, off.data(), off.size() * sizeof(int32_t));
+  if (nbr_idx) std::memcpy(nbr_idx, idx.data(), idx.size() * sizeof(int32_t));
+  return UG_OK;
+}
+
+int ug_visible_pairs(const ug_geom* g, int64_t* hr_hr, int64_t* hr_lr, int64_t* lr_lr) {
+  int st = validate(g);
+  if (st != UG_OK) return st;
+  std::vector<int32_t> off, idx;
+  build_neighbours(*g, off, idx);
+  const int64_t T = (int64_t)g->win_h * g->win_w;
+  const int64_t N = (int64_t)g->grid_h * g->grid_w, L = (int64_t)g->lr_h * g->lr_w;
+  if (hr_hr) *hr_hr = (int64_t)idx.size() * T * T;
+  if (hr_lr) *hr_lr = N * L;
+  if (lr_lr) *lr_lr = L * L;
+  return UG_OK;
+}
+
+const char* ug_status_string(int s) {
+  switch (s) {
+    case UG_OK: return "ok";
+    case UG_ERR_INVALID_ARG: return "invalid argument";
+    case UG_ERR_UNSUPPORTED: return "unsupported geometry";
+    case UG_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case UG_ERR_ALIAS: return "output overlaps an input";
+    case UG_ERR_CUDA: return "CUDA error";
+    case UG_ERR_TIMEOUT: return "device-side wait timed out";
+    case UG_ERR_NO_MEMORY: return "out of memory";
+    default: return "unknown status";
+  }
+}
+
+int ug_plan_create(const ug_geom* g, ug_plan** out) {
+  if (!out) return UG_ERR_INVALID_ARG;
+  *out = nullptr;
+  int st = validate(g);
+  if (st != UG_OK) return st;
+  ug_plan* p = new (std::nothrow) ug_plan();
+  if (!p) return UG_ERR_NO_MEMORY;
+  p->g = *g;
+  p->N = (int64_t)g->grid_h * g->grid_w;
+  p->L = (int64_t)g->lr_h * g->lr_w;
+  p->T = (int64_t)g->win_h * g->win_w;
+  p->nwy = g->grid_h / g->win_h;
+  p->nwx = g->grid_w / g->win_w;
+  p->scale = g->softmax_scale > 0.0f ? g->softmax_scale : (float)(1.0 / std::sqrt((double)g->head_dim));
+  p->wait_timeout_ns = kDefaultWaitTimeoutNs;
+  p->d_mem = nullptr;
+  try {
+    build_perm(*g, p->perm);
+    build_neighbours(*g, p->nbr_off, p->nbr_idx);
+    build_attention_lists(*g, p->nbr_off, p->nbr_idx, p->qtiles, p->kvlist, &p->n_hr_ctas,
+                          &p->n_lr_ctas);
+    std::vector<float> tables;
+    build_rope_tables(*g, p->rope, tables);
+    // One device block: [err (256 B)] [rope tables] [qtiles] [kvlist]
+    const size_t a_err = 0;
+    const size_t a_rope = 256;
+    const size_t a_qt = (a_rope + tables.size() * sizeof(float) + 255) / 256 * 256;
+    const size_t a_kv = (a_qt + p->qtiles.size() * sizeof(QTile) + 255) / 256 * 256;
+    const size_t total = a_kv + std::max<size_t>(1, p->kvlist.size()) * sizeof(uint32_t);
+    if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return UG_ERR_CUDA; }
+    if (cudaMalloc(&p->d_mem, total) != cudaSuccess) {
+      cudaGetLastError();
+      delete p;
+      return UG_ERR_NO_MEMORY;
+    }
+    char* base = static_cast<char*>(p->d_mem);
+    p->d_err = reinterpret_cast<int*>(base + a_err);
+    p->d_rope = reinterpret_cast<float*>(base + a_rope);
+    p->d_qtiles = reinterpret_cast<QTile*>(base + a_qt);
+    p->d_kvlist = reinterpret_cast<uint32_t*>(base + a_kv);
+    std::vector<char> host(total, 0);
+    std::memcpy(host.data() + a_rope, tables.data(), tables.size() * sizeof(float));
+    std::memcpy(host.data() + a_qt, p->qtiles.data(), p->qtiles.size() * sizeof(QTile));
+    std::memcpy(host.data() + a_kv, p->kvlist.data(), p->kvlist.size() * sizeof(uint32_t));
+    if (cudaMemcpy(p->d_mem, host.data(), total, cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(p->d_mem);
+      delete p;
+      return UG_ERR_CUDA;
+    }
+  } catch (const std::bad_alloc&) {
+    if (p->d_mem) cudaFree(p->d_mem);
+    delete p;
+    return UG_ERR_NO_MEMORY;
+  }
+  *out = p;
+  return UG_OK;
+}
+
+int ug_plan_destroy(ug_plan* p) {
+  if (!p) return UG_OK;
+  int st = UG_OK;
+  if (p->d_mem) {
+    if (cudaDeviceSynchronize() != cudaSuccess) st = UG_ERR_CUDA;
+    if (cudaFree(p->d_mem) != cudaSuccess) st = UG_ERR_CUDA;
+  }
+  delete p;
+  return st;
+}
+
+int ug_get_index_maps(const ug_plan* p, int32_t* perm, int32_t* nbr_off, int32_t* nbr_idx) {
+  if (!p) return UG_ERR_INVALID_ARG;
+  if (perm) std::memcpy(perm, p->perm.data(), p->perm.size() * sizeof(int32_t));
+  if (nbr_off) std::memcpy(nbr_off, p->nbr_off.data(), p->nbr_off.size() * sizeof(int32_t));
+  if (nbr_idx) std::memcpy(nbr_idx, p->nbr_idx.data(), p->nbr_idx.size() * sizeof(int32_t));
+  return UG_OK;
+}
+
+static int permute_common(const ug_plan* p, const void* src, void* dst, bool inverse, void* s) {
+  if (!p || !src || !dst) return UG_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return UG_ERR_ALIGNMENT;
+  const int64_t n = hr_bytes(p);
+  if (overlap(src, n, dst, n)) return UG_ERR_ALIAS;
+  return launch_permute(p, src, dst, inverse, as_stream(s));
+}
+
+int ug_permute_window_first(const ug_plan* p, const void* src_raster, void* dst_wf, void* s) {
+  return permute_common(p, src_raster, dst_wf, false, s);
+}
+
+int ug_unpermute(const ug_plan* p, const void* src_wf, void* dst_raster, void* s) {
+  return permute_common(p, src_wf, dst_raster, true, s);
+}
+
+int ug_rope_2d(const ug_plan* p, const void* x, void* y, int token_set, void* s) {
+  if (!p || !x || !y) return UG_ERR_INVALID_ARG;
+  if (token_set != UG_HR_WINDOW_FIRST && token_set != UG_HR_RASTER && token_set != UG_LR)
+    return UG_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return UG_ERR_ALIGNMENT;
+  const int64_t n = token_set == UG_LR ? lr_bytes(p) : hr_bytes(p);
+  if (n == 0) return UG_OK;
+  if (x != y && overlap(x, n, y, n)) return UG_ERR_ALIAS;
+  return launch_rope(p, x, y, token_set, as_stream(s));
+}
+
+int ug_hier_local_attn_fwd(const ug_plan* p, const void* q_hr, const void* k_hr,
+                           const void* v_hr, const void* q_lr, const void* k_lr,
+                           const void* v_lr, void* o_hr, void* o_lr, float* lse, void* s) {
+  if (!p || !q_hr || !k_hr || !v_hr || !o_hr) return UG_ERR_INVALID_ARG;
+  if (p->L > 0 && (!q_lr || !k_lr || !v_lr || !o_lr)) return UG_ERR_INVALID_ARG;
+  if (p->g.head_dim != 64 && p->g.head_dim != 128) return UG_ERR_UNSUPPORTED;
+  const void* ins[6] = {q_hr, k_hr, v_hr, q_lr, k_lr, v_lr};
+  for (const void* a : ins)
+    if (a && !aligned16(a)) return UG_ERR_ALIGNMENT;
+  if (!aligned16(o_hr) || (o_lr && !aligned16(o_lr)) || (lse && !aligned16(lse)))
+    return UG_ERR_ALIGNMENT;
+  const int64_t nh = hr_bytes(p), nl = lr_bytes(p);
+  const int64_t nlse = lse ? (int64_t)p->g.batch * p->g.heads * (p->N + p->L) * 4 : 0;
+  const int64_t sizes[6] = {nh, nh, nh, nl, nl, nl};
+  for (int i = 0; i < 6; ++i) {
+    if (overlap(o_hr, nh, ins[i], sizes[i]) || overlap(o_lr, nl, ins[i], sizes[i]) ||
+        overlap(lse, nlse, ins[i], sizes[i]))
+      return UG_ERR_ALIAS;
+  }
+  if (overlap(o_hr, nh, o_lr, nl) || overlap(o_hr, nh, lse, nlse) || overlap(o_lr, nl, lse, nlse))
+    return UG_ERR_ALIAS;
+  return launch_attention(p, q_hr, k_hr, v_hr, p->L ? q_lr : nullptr, p->L ? k_lr : nullptr,
+                          p->L ? v_lr : nullptr, o_hr, p->L ? o_lr : nullptr, lse,
+                          as_stream(s));
+}
+
+int64_t ug_layer_workspace_bytes(const ug_plan* p) {
+  if (!p) return -1;
+  auto up = [](int64_t n) { return (n + 255) / 256 * 256; };
+  return 4 * up(hr_bytes(p)) + 2 * up(lr_bytes(p));
+}
+
+int ug_layer_fwd(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+                 const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr, void* o_lr,
+                 float* lse, void* workspace, int64_t workspace_bytes, void* s) {
+  if (!p || !workspace) return UG_ERR_INVALID_ARG;
+  if (workspace_bytes < ug_layer_workspace_bytes(p)) return UG_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return UG_ERR_ALIGNMENT;
+  if (!q_hr || !k_hr || !v_hr || !o_hr) return UG_ERR_INVALID_ARG;
+  if (p->L > 0 && (!q_lr || !k_lr || !v_lr || !o_lr)) return UG_ERR_INVALID_ARG;
+  if (p->g.head_dim != 64 && p->g.head_dim != 128) return UG_ERR_UNSUPPORTED;
+  const int64_t ws = ug_layer_workspace_bytes(p);
+  const void* ins[6] = {q_hr, k_hr, v_hr, q_lr, k_lr, v_lr};
+  const int64_t nh = hr_bytes(p), nl = lr_bytes(p);
+  const int64_t sizes[6] = {nh, nh, nh, nl, nl, nl};
+  for (int i = 0; i < 6; ++i)
+    if (overlap(workspace, ws, ins[i], sizes[i])) return UG_ERR_ALIAS;
+  auto up = [](int64_t n) { return (n + 255) / 256 * 256; };
+  char* w = static_cast<char*>(workspace);
+  void* q_wf = w;
+  void* k_wf = w + up(nh);
+  void* v_wf = w + 2 * up(nh);
+  void* o_wf = w + 3 * up(nh);
+  void* q_lr_r = w + 4 * up(nh);
+  void* k_lr_r = w + 4 * up(nh) + up(nl);
+  if (overlap(workspace, ws, o_hr, nh) || overlap(workspace, ws, o_lr, nl))
+    return UG_ERR_ALIAS;
+  int st;
+  if ((st = ug_permute_window_first(p, q_hr, q_wf, s)) != UG_OK) return st;
+  if ((st = ug_permute_window_first(p, k_hr, k_wf, s)) != UG_OK) return st;
+  if ((st = ug_permute_window_first(p, v_hr, v_wf, s)) != UG_OK) return st;
+  if ((st = ug_rope_2d(p, q_wf, q_wf, UG_HR_WINDOW_FIRST, s)) != UG_OK) return st;
+  if ((st = ug_rope_2d(p, k_wf, k_wf, UG_HR_WINDOW_FIRST, s)) != UG_OK) return st;
+  if (p->L > 0) {
+    if ((st = ug_rope_2d(p, q_lr, q_lr_r, UG_LR, s)) != UG_OK) return st;
+    if ((st = ug_rope_2d(p, k_lr, k_lr_r, UG_LR, s)) != UG_OK) return st;
+  }
+  if ((st = ug_hier_local_attn_fwd(p, q_wf, k_wf, v_wf, q_lr_r, k_lr_r, v_lr, o_wf, o_lr, lse,
+                                   s)) != UG_OK)
+    return st;
+  return ug_unpermute(p, o_wf, o_hr, s);
+}
+
+int ug_check_error(const ug_plan* p, void* s) {
+  if (!p) return UG_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(as_stream(s)) != cudaSuccess) return UG_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, p->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return UG_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p->d_err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return UG_ERR_CUDA;
+    return h;
+  }
+  if (cudaGetLastError() != cudaSuccess) return UG_ERR_CUDA;
+  return UG_OK;
+}
+
+}  // extern "C"

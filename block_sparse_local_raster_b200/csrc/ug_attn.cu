@@ -1,0 +1,679 @@
+// Block-sparse joint-softmax attention of the hierarchical local attention
+// layer on B200 (sm_100a): tcgen05 MMA with TMEM accumulators, TMA loads,
+// mbarrier pipeline, warp specialisation.
+//
+// What it computes (UltraGen-ar §2.ب "Attention Masking"; UltraGen-es §2,
+// guidance item; UltraGen-it §2): a high-res query of window w attends, under
+// one softmax, to the high-res keys of every window within Chebyshev distance
+// `radius` of w and to every low-res key; a low-res query attends to the
+// low-res keys only.  High-res tensors arrive window-first (UltraGen-fr §2.A),
+// so a window is a contiguous run of keys and the mask is block structured:
+// a host-built list names, per 256-row query CTA, the 128-key blocks that
+// hold visible keys (every other block is never loaded), and flags the few
+// blocks that need a per-pair test (ragged ends, windows that straddle a
+// block).
+//
+// CTA layout (320 threads):
+//   warps 0-3  softmax for query tile 0 (rows 0..127 of the CTA)
+//   warps 4-7  softmax for query tile 1 (rows 128..255)
+//   warp 8     TMA producer: Q once, then K_j, V_j into a 3-slot ring
+//   warp 9     TMEM allocation and the tcgen05.mma issuer
+// TMEM (512 columns x 128 lanes x 32 bit): S0 [0,128) S1 [128,256)
+//   O0 [256, 256+D) O1 [384, 384+D).  One TMEM lane = one query row, so the
+//   row max and row sum are in-thread (no shuffles needed).
+// Shared memory: Q0 Q1, K/V ring, P0 P1 (bf16 probabilities, K-major, 128-byte
+//   swizzle, the A operand of O += P V).
+// Pipeline per key block j (tiles ping-pong so that one softmax overlaps the
+//   other tile's MMAs):  S0=Q0 K_j^T, S1=Q1 K_j^T | softmax0(j) | O0+=P0 V_j,
+//   S0=Q0 K_{j+1}^T | softmax1(j) | O1+=P1 V_j, S1=Q1 K_{j+1}^T | ...
+// Online softmax in the log2 domain with lazy rescaling: the running
+// reference max moves (and O, l are rescaled) only when a block's max exceeds
+// it by more than 8 (a factor 256), so probabilities stay <= 256 and O is
+// rarely touched.
+//
+// Every wait is bounded (globaltimer); on expiry a thread records
+// UG_ERR_TIMEOUT in the plan's error word, raises a CTA-wide abort flag and
+// every role unwinds: the producer waits (bounded) for its loads in flight,
+// the MMA warp for its MMAs, then TMEM is freed and the CTA exits.
+#include <cstdint>
+#include <cstring>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ug_internal.h"
+
+namespace ug {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kStages = 3;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+#define kNegInf __int_as_float(0xff800000)
+
+template <int D>
+struct Layout {
+  static constexpr int kTileBytes = kRowsPerTile * D * 2;     // Q tile, K or V tile
+  static constexpr int kPBytes = kRowsPerTile * kKeysPerBlock * 2;
+  static constexpr int kQ = 0;
+  static constexpr int kKV = kQ + kTilesPerCta * kTileBytes;
+  static constexpr int kP = kKV + kStages * kTileBytes;
+  static constexpr int kBar = kP + kTilesPerCta * kPBytes;
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 3 * kTilesPerCta + 1;
+  static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base (u32), abort flag (u32)
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+};
+
+struct AttnParams {
+  const QTile* qtiles;
+  const uint32_t* kvlist;
+  __nv_bfloat16* o_hr;
+  __nv_bfloat16* o_lr;
+  float* lse;
+  int* err;
+  int64_t timeout_ns;
+  int32_t N, L, T, nwx, radius, heads;
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+// ---------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on a barrier phase.  Gives up when the CTA's abort flag is up
+// (unless ignore_abort) or after timeout_ns; on a timeout it records the
+// status and raises the abort flag.  Returns true when the phase completed.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                       int* err, int64_t timeout_ns, bool ignore_abort) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (!ignore_abort && *abort) return false;
+      if ((int64_t)(globaltimer() - t0) > timeout_ns) {
+        atomicCAS(err, 0, (int)UG_ERR_TIMEOUT);
+        *abort = 1u;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int32_t c0,
+                                            int32_t c1, int32_t c2, int32_t c3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100
+// descriptor version 1.  lbo/sbo in bytes.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M = 128.
+__host__ __device__ constexpr uint32_t instr_desc(int n, bool b_mn_major) {
+  return (1u << 4)                  // D format: f32
+         | (1u << 7)                // A format: bf16
+         | (1u << 10)               // B format: bf16
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(n >> 3) << 17)
+         | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// ---------------------------------------------------------------- the kernel
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    hier_attn_kernel(const __grid_constant__ CUtensorMap tm_q_hr,
+                     const __grid_constant__ CUtensorMap tm_k_hr,
+                     const __grid_constant__ CUtensorMap tm_v_hr,
+                     const __grid_constant__ CUtensorMap tm_q_lr,
+                     const __grid_constant__ CUtensorMap tm_k_lr,
+                     const __grid_constant__ CUtensorMap tm_v_lr, const AttnParams P) {
+  using Lay = Layout<D>;
+  constexpr int kRegions = D / 64;  // 128-byte swizzle spans 64 bf16 columns
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + Lay::kBar;
+  const uint32_t q_full = bar0;
+  auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + kStages + s); };
+  auto s_full = [&](int t) { return bar0 + 8u * (1 + 2 * kStages + t); };
+  auto p_full = [&](int t) { return bar0 + 8u * (1 + 2 * kStages + 2 + t); };
+  auto o_done = [&](int t) { return bar0 + 8u * (1 + 2 * kStages + 4 + t); };
+  const uint32_t drain = bar0 + 8u * (1 + 2 * kStages + 6);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
+  volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + Lay::kMisc + 4);
+  int* const err = P.err;
+  const int64_t timeout_ns = P.timeout_ns;
+  // Single-thread roles wait alone; the softmax warps agree on the outcome so
+  // that the warp-collective tcgen05 loads that follow never run diverged.
+  auto wait1 = [&](uint32_t bar, uint32_t par) {
+    return mbar_wait(bar, par, abort, err, timeout_ns, false);
+  };
+  auto drain_wait = [&](uint32_t bar, uint32_t par) {
+    return mbar_wait(bar, par, abort, err, timeout_ns, true);
+  };
+  auto wait_warp = [&](uint32_t bar, uint32_t par) {
+    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, par, abort, err, timeout_ns, false)) != 0;
+  };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const QTile qt = P.qtiles[blockIdx.x];
+  const int head = blockIdx.y;
+  const int b = blockIdx.z;
+  const int nblk = qt.list_len;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int t = 0; t < kTilesPerCta; ++t) {
+      mbar_init(s_full(t), 1);
+      mbar_init(p_full(t), kRowsPerTile);
+      mbar_init(o_done(t), 1);
+    }
+    mbar_init(drain, 1);
+    // A CTA that starts after another one gave up does no work.
+    *abort = *reinterpret_cast<volatile int*>(err) != 0 ? 1u : 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    prefetch_map(&tm_q_hr);
+    prefetch_map(&tm_k_hr);
+    prefetch_map(&tm_v_hr);
+    if (P.L > 0) {
+      prefetch_map(&tm_q_lr);
+      prefetch_map(&tm_k_lr);
+      prefetch_map(&tm_v_lr);
+    }
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = *abort != 0u;
+
+  if (skip) {
+    // nothing issued: fall through to the teardown
+  } else if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const CUtensorMap* mq = qt.lowres ? &tm_q_lr : &tm_q_hr;
+      mbar_expect_tx(q_full, kTilesPerCta * Lay::kTileBytes);
+      for (int t = 0; t < kTilesPerCta; ++t)
+        for (int r = 0; r < kRegions; ++r)
+          tma_load_4d(sbase + Lay::kQ + t * Lay::kTileBytes + r * kRowsPerTile * 128, mq, r * 64,
+                      head, qt.q0 + t * kRowsPerTile, b, q_full);
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < nblk && ok; ++j) {
+        const uint32_t e = P.kvlist[qt.list_off + j];
+        const bool lr = (e & kBlockLowres) != 0;
+        const int k0 = (int)(e & kBlockIndexMask) * kKeysPerBlock;
+        for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
+          const CUtensorMap* m = kv == 0 ? (lr ? &tm_k_lr : &tm_k_hr) : (lr ? &tm_v_lr : &tm_v_hr);
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (!wait1(kv_empty(s), ph ^ 1u)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(kv_full(s), Lay::kTileBytes);
+          for (int r = 0; r < kRegions; ++r)
+            tma_load_4d(sbase + Lay::kKV + s * Lay::kTileBytes + r * kKeysPerBlock * 128, m,
+                        r * 64, head, k0, b, kv_full(s));
+        }
+      }
+      // Loads still in flight land before the CTA may exit.  The last
+      // kStages loads each own a distinct slot, and no later phase of that
+      // slot exists, so waiting for that phase is unambiguous.
+      for (int i = (it > kStages ? it - kStages : 0); i < it; ++i)
+        drain_wait(kv_full(i % kStages), (uint32_t)(i / kStages) & 1u);
+      drain_wait(q_full, 0);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = instr_desc(kKeysPerBlock, false);
+      constexpr uint32_t kIdO = instr_desc(D, true);
+      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + 128u};
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = sbase + Lay::kQ + t * Lay::kTileBytes;
+        const uint32_t ka = sbase + Lay::kKV + slot * Lay::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * (kRowsPerTile * 128) + (kk % 4) * 32;
+          mma_bf16(tS[t], smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024), kIdS,
+                   kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t pa = sbase + Lay::kP + t * Lay::kPBytes;
+        const uint32_t va = sbase + Lay::kKV + slot * Lay::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kKeysPerBlock / 16; ++kk) {
+          const uint32_t aoff = (kk / 4) * (kRowsPerTile * 128) + (kk % 4) * 32;
+          const uint32_t boff = kk * 16 * 128;
+          mma_bf16(tO[t], smem_desc(pa + aoff, 16, 1024),
+                   smem_desc(va + boff, kKeysPerBlock * 128, 1024), kIdO, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = wait1(q_full, 0);
+      if (ok) ok = wait1(kv_full(0), 0);
+      if (ok) {
+        fence_after();
+        issue_s(0, 0);
+        mma_commit(s_full(0));
+        issue_s(1, 0);
+        mma_commit(s_full(1));
+        mma_commit(kv_empty(0));
+      }
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int itv = 2 * j + 1, itk = 2 * j + 2;
+        const int sv = itv % kStages, sk = itk % kStages;
+        if (!(ok = wait1(kv_full(sv), (uint32_t)(itv / kStages) & 1u))) break;
+        if (!(ok = wait1(p_full(0), (uint32_t)j & 1u))) break;
+        fence_after();
+        issue_pv(0, sv, j > 0);
+        mma_commit(o_done(0));
+        const bool more = j + 1 < nblk;
+        if (more) {
+          if (!(ok = wait1(kv_full(sk), (uint32_t)(itk / kStages) & 1u))) break;
+          fence_after();
+          issue_s(0, sk);
+          mma_commit(s_full(0));
+        }
+        if (!(ok = wait1(p_full(1), (uint32_t)j & 1u))) break;
+        fence_after();
+        issue_pv(1, sv, j > 0);
+        mma_commit(o_done(1));
+        mma_commit(kv_empty(sv));
+        if (more) {
+          issue_s(1, sk);
+          mma_commit(s_full(1));
+          mma_commit(kv_empty(sk));
+        }
+      }
+      // Every MMA issued above completes before TMEM may be freed.
+      mma_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2;               // query tile
+    const int row = (warp & 3) * 32 + lane;  // TMEM lane = row in tile
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (t ? 128u : 0u);
+    const uint32_t tO = tmem + lane_base + 256u + (t ? 128u : 0u);
+    uint8_t* p_row = smem + Lay::kP + t * Lay::kPBytes + row * 128;
+    const int tok = qt.q0 + t * kRowsPerTile + row;  // query token in its tensor
+    const int q_w = tok / P.T;
+    const int q_wy = q_w / P.nwx, q_wx = q_w - (q_w / P.nwx) * P.nwx;
+    float m_ref = kNegInf;  // reference max (log2 units) of the O/l accumulators
+    float l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nblk; ++j) {
+      const uint32_t e = P.kvlist[qt.list_off + j];
+      if (!(ok = wait_warp(s_full(t), (uint32_t)j & 1u))) break;
+      fence_after();
+      float s[kKeysPerBlock];
+#pragma unroll
+      for (int c = 0; c < kKeysPerBlock / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
+      tmem_ld_wait();
+      if (e & kBlockMasked) {
+        const int k0 = (int)(e & kBlockIndexMask) * kKeysPerBlock;
+        if (e & kBlockLowres) {
+#pragma unroll
+          for (int i = 0; i < kKeysPerBlock; ++i)
+            if (k0 + i >= P.L) s[i] = kNegInf;
+        } else {
+          // Visibility changes only at window boundaries: test each key
+          // window met in the block once, then mask its run of keys.
+          int i0 = 0;
+          while (i0 < kKeysPerBlock) {
+            const int k = k0 + i0;
+            const int kw = k / P.T;
+            const int run = min(kKeysPerBlock, (kw + 1) * P.T - k0);
+            const int kwy = kw / P.nwx, kwx = kw - (kw / P.nwx) * P.nwx;
+            const bool vis = abs(kwy - q_wy) <= P.radius && abs(kwx - q_wx) <= P.radius;
+            const int lim = vis ? min(run, P.N - k0) : i0;  // keys [i0, lim) stay
+#pragma unroll
+            for (int i = 0; i < kKeysPerBlock; ++i)
+              if (i >= i0 && i < run && i >= lim) s[i] = kNegInf;
+            i0 = run;
+          }
+        }
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < kKeysPerBlock; ++i) mx = fmaxf(mx, s[i]);
+      const float m_blk = mx * P.scale_log2;
+      const bool rescale = m_blk > m_ref + kRescaleThreshold;
+      const float m_new = rescale ? m_blk : m_ref;
+      const float alpha = rescale ? fast_exp2(m_ref - m_new) : 1.0f;
+      const float m_use = m_new == kNegInf ? 0.0f : m_new;
+      m_ref = m_new;
+      if (j > 0) {
+        // O += P V of the previous block must be complete before its P
+        // buffer is overwritten and before O is rescaled.  It was issued
+        // ahead of this block's S, so it has normally retired already.
+        if (!(ok = wait_warp(o_done(t), (uint32_t)(j - 1) & 1u))) break;
+        fence_after();
+        if (__any_sync(0xFFFFFFFFu, rescale)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            float o[16];
+            tmem_ld16(tO + c * 16, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] *= alpha;
+            tmem_st16(tO + c * 16, o);
+          }
+          tmem_st_wait();
+        }
+      }
+      // p = 2^(s*scale*log2e - m): row sum in fp32, P row to shared memory
+      // as bf16, K-major with the 128-byte swizzle (16-byte chunk c of a
+      // 128-byte row lands at chunk c ^ (row % 8)).
+      float rowsum = 0.0f;
+#pragma unroll
+      for (int c = 0; c < kKeysPerBlock / 8; ++c) {
+        float p[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          p[i] = fast_exp2(fmaf(s[8 * c + i], P.scale_log2, -m_use));
+          rowsum += p[i];
+        }
+        const uint4 v = make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
+                                   pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
+        const int region = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4*>(p_row + region * (kRowsPerTile * 128) + ((cc ^ (row & 7)) << 4)) = v;
+      }
+      l = l * alpha + rowsum;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      fence_before();
+      mbar_arrive(p_full(t));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = wait_warp(o_done(t), (uint32_t)(nblk - 1) & 1u);
+    if (ok) {
+      fence_after();
+      const int ntok = qt.lowres ? P.L : P.N;
+      const bool valid = tok < ntok;
+      const float inv_l = 1.0f / l;
+      __nv_bfloat16* dst = (qt.lowres ? P.o_lr : P.o_hr) +
+                           (((int64_t)b * ntok + tok) * P.heads + head) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v = make_uint4(pack_bf16(o[i] * inv_l, o[i + 1] * inv_l),
+                                 pack_bf16(o[i + 2] * inv_l, o[i + 3] * inv_l),
+                                 pack_bf16(o[i + 4] * inv_l, o[i + 5] * inv_l),
+                                 pack_bf16(o[i + 6] * inv_l, o[i + 7] * inv_l));
+            *reinterpret_cast<uint4*>(dst + c * 32 + i) = v;
+          }
+        }
+      }
+      if (valid && P.lse) {
+        const float lse = (m_ref + __log2f(l)) * 0.69314718055994531f;
+        P.lse[((int64_t)b * P.heads + head) * (P.N + P.L) + (qt.lowres ? P.N : 0) + tok] = lse;
+      }
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [B, n_tok, heads, D] bf16 -> box of 64 channels x 1 head x 128 tokens.
+bool make_map(CUtensorMap* m, const void* base, int64_t B, int64_t n_tok, int heads, int D) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)heads,
+                              (cuuint64_t)std::max<int64_t>(n_tok, 1), (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2,
+                                 (cuuint64_t)std::max<int64_t>(n_tok, 1) * heads * D * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)kRowsPerTile, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch_d(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+             const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr, void* o_lr,
+             float* lse, cudaStream_t st) {
+  const int64_t B = p->g.batch;
+  const int H = p->g.heads;
+  CUtensorMap m[6];
+  const void* lrs[3] = {q_lr ? q_lr : q_hr, k_lr ? k_lr : k_hr, v_lr ? v_lr : v_hr};
+  const int64_t nl = p->L > 0 ? p->L : p->N;
+  if (!make_map(&m[0], q_hr, B, p->N, H, D) || !make_map(&m[1], k_hr, B, p->N, H, D) ||
+      !make_map(&m[2], v_hr, B, p->N, H, D) || !make_map(&m[3], lrs[0], B, nl, H, D) ||
+      !make_map(&m[4], lrs[1], B, nl, H, D) || !make_map(&m[5], lrs[2], B, nl, H, D))
+    return UG_ERR_CUDA;
+  AttnParams P;
+  P.qtiles = p->d_qtiles;
+  P.kvlist = p->d_kvlist;
+  P.o_hr = static_cast<__nv_bfloat16*>(o_hr);
+  P.o_lr = static_cast<__nv_bfloat16*>(o_lr);
+  P.lse = lse;
+  P.err = p->d_err;
+  P.timeout_ns = p->wait_timeout_ns;
+  P.N = (int32_t)p->N;
+  P.L = (int32_t)p->L;
+  P.T = (int32_t)p->T;
+  P.nwx = p->nwx;
+  P.radius = p->g.radius;
+  P.heads = H;
+  P.scale_log2 = p->scale * 1.4426950408889634f;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(hier_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Layout<D>::kAlloc) != cudaSuccess)
+      return UG_ERR_CUDA;
+    attr_set = true;
+  }
+  const dim3 grid((unsigned)p->qtiles.size(), (unsigned)H, (unsigned)B);
+  hier_attn_kernel<D><<<grid, kThreads, Layout<D>::kAlloc, st>>>(m[0], m[1], m[2], m[3], m[4],
+                                                                  m[5], P);
+  return cudaGetLastError() == cudaSuccess ? UG_OK : UG_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+                     const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
+                     void* o_lr, float* lse, cudaStream_t st) {
+  if (p->g.head_dim == 128)
+    return launch_d<128>(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, st);
+  if (p->g.head_dim == 64)
+    return launch_d<64>(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, st);
+  return UG_ERR_UNSUPPORTED;
+}
+
+}  // namespace ug

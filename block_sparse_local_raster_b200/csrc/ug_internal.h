@@ -1,0 +1,92 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "ug.h"
+
+namespace ug {
+
+// Attention tiling: a CTA owns 256 consecutive query rows of one token set
+// (two 128-row tiles, one TMEM lane per row) and walks a list of 128-key
+// blocks.
+constexpr int kRowsPerTile = 128;
+constexpr int kTilesPerCta = 2;
+constexpr int kRowsPerCta = kRowsPerTile * kTilesPerCta;
+constexpr int kKeysPerBlock = 128;
+
+// One query CTA of the attention: which token set its rows belong to, its
+// first row, and its slice of the key-block list.
+struct QTile {
+  int32_t lowres;    // 0: high-res rows (window-first), 1: low-res rows
+  int32_t q0;        // first query token of the CTA inside its tensor
+  int32_t list_off;  // first entry in the key-block list
+  int32_t list_len;  // number of key blocks (>= 1)
+};
+
+// Key-block list entry: block index (keys [128*idx, 128*idx + 128) of its
+// tensor), whether it lies in the low-res tensor, and whether some
+// (query, key) pair inside it is invisible or out of range so that the
+// kernel must test each pair.
+constexpr uint32_t kBlockIndexMask = (1u << 29) - 1;
+constexpr uint32_t kBlockLowres = 1u << 29;
+constexpr uint32_t kBlockMasked = 1u << 30;
+
+// Offsets (in floats) of the RoPE tables inside the plan's table buffer.
+// Each table is [coordinate][pair k], fp32; cos and sin separately.
+struct RopeTables {
+  int64_t hr_y_cos, hr_y_sin, hr_x_cos, hr_x_sin;
+  int64_t lr_y_cos, lr_y_sin, lr_x_cos, lr_x_sin;
+  int64_t total;
+};
+
+// Upper bound of a device-side wait before a kernel gives up (ns).
+constexpr int64_t kDefaultWaitTimeoutNs = 2000000000ll;
+
+}  // namespace ug
+
+struct ug_plan {
+  ug_geom g;
+  int64_t N, L, T;   // high-res tokens, low-res tokens, tokens per window
+  int32_t nwy, nwx;  // windows per axis
+  float scale;       // softmax scale actually used
+  int device;
+
+  std::vector<int32_t> perm, nbr_off, nbr_idx;
+  std::vector<ug::QTile> qtiles;
+  std::vector<uint32_t> kvlist;
+  int32_t n_hr_ctas, n_lr_ctas;
+  ug::RopeTables rope;
+
+  void* d_mem;             // one device allocation holding everything below
+  float* d_rope;           // RoPE tables
+  ug::QTile* d_qtiles;     // attention query CTAs
+  uint32_t* d_kvlist;      // attention key-block lists
+  int* d_err;              // first device-side error status (0 = none)
+  int64_t wait_timeout_ns;
+};
+
+namespace ug {
+
+// Host plan pieces (ug_plan.cu).
+int validate(const ug_geom* g);
+void build_perm(const ug_geom& g, std::vector<int32_t>& perm);
+void build_neighbours(const ug_geom& g, std::vector<int32_t>& off, std::vector<int32_t>& idx);
+void build_attention_lists(const ug_geom& g, const std::vector<int32_t>& nbr_off,
+                           const std::vector<int32_t>& nbr_idx, std::vector<QTile>& qtiles,
+                           std::vector<uint32_t>& kvlist, int32_t* n_hr_ctas, int32_t* n_lr_ctas);
+void build_rope_tables(const ug_geom& g, RopeTables& off, std::vector<float>& data);
+
+// Kernel launchers (one .cu each).  Arguments are already checked.
+int launch_permute(const ug_plan* p, const void* src, void* dst, bool inverse, cudaStream_t s);
+int launch_rope(const ug_plan* p, const void* x, void* y, int token_set, cudaStream_t s);
+int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+                     const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
+                     void* o_lr, float* lse, cudaStream_t s);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace ug

@@ -1,0 +1,265 @@
+"""Thin ctypes binding of libug (include/ug.h): argument marshalling only.
+
+Every function keeps the C name.  Tensors are torch tensors (device memory
+and streams come from PyTorch); every step of the layer runs in the
+library's CUDA kernels.  If libug.so is missing the first call raises; there
+is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libug.so")
+
+UG_OK = 0
+UG_ERR_INVALID_ARG = 1
+UG_ERR_UNSUPPORTED = 2
+UG_ERR_ALIGNMENT = 3
+UG_ERR_ALIAS = 4
+UG_ERR_CUDA = 5
+UG_ERR_TIMEOUT = 6
+UG_ERR_NO_MEMORY = 7
+
+UG_HR_WINDOW_FIRST = 0
+UG_HR_RASTER = 1
+UG_LR = 2
+
+# Every symbol include/ug.h declares.
+EXPORTS = (
+    "ug_geom_validate", "ug_index_map_sizes", "ug_build_index_maps", "ug_visible_pairs",
+    "ug_status_string", "ug_plan_create", "ug_plan_destroy", "ug_get_index_maps",
+    "ug_permute_window_first", "ug_unpermute", "ug_rope_2d", "ug_hier_local_attn_fwd",
+    "ug_layer_workspace_bytes", "ug_layer_fwd", "ug_check_error",
+)
+
+
+class UgError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class ug_geom(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+        ("win_h", ctypes.c_int32), ("win_w", ctypes.c_int32), ("radius", ctypes.c_int32),
+        ("lr_h", ctypes.c_int32), ("lr_w", ctypes.c_int32), ("rho", ctypes.c_double),
+        ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("rope_dim_y", ctypes.c_int32), ("rope_dim_x", ctypes.c_int32),
+        ("rope_theta", ctypes.c_double), ("softmax_scale", ctypes.c_float),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libug.so once (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m block_sparse_local_raster_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I32, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    G = ctypes.POINTER(ug_geom)
+    pi32 = ctypes.POINTER(ctypes.c_int32)
+    pi64 = ctypes.POINTER(ctypes.c_int64)
+    sig = {
+        "ug_geom_validate": (I32, [G]),
+        "ug_index_map_sizes": (I32, [G, pi64, pi64, pi64]),
+        "ug_build_index_maps": (I32, [G, pi32, pi32, pi32]),
+        "ug_visible_pairs": (I32, [G, pi64, pi64, pi64]),
+        "ug_status_string": (ctypes.c_char_p, [I32]),
+        "ug_plan_create": (I32, [G, ctypes.POINTER(P)]),
+        "ug_plan_destroy": (I32, [P]),
+        "ug_get_index_maps": (I32, [P, pi32, pi32, pi32]),
+        "ug_permute_window_first": (I32, [P, P, P, P]),
+        "ug_unpermute": (I32, [P, P, P, P]),
+        "ug_rope_2d": (I32, [P, P, P, I32, P]),
+        "ug_hier_local_attn_fwd": (I32, [P, P, P, P, P, P, P, P, P, P, P]),
+        "ug_layer_workspace_bytes": (I64, [P]),
+        "ug_layer_fwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I64, P]),
+        "ug_check_error": (I32, [P, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().ug_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != UG_OK:
+        raise UgError(status, what)
+
+
+def make_geom(**kw) -> ug_geom:
+    g = ug_geom()
+    for name, _ in ug_geom._fields_:
+        setattr(g, name, kw.get(name, 0))
+    return g
+
+
+def geom_validate(g: ug_geom) -> int:
+    return lib().ug_geom_validate(ctypes.byref(g))
+
+
+def build_index_maps(g: ug_geom):
+    """(perm, nbr_off, nbr_idx) as int32 numpy arrays (host only)."""
+    n = [ctypes.c_int64() for _ in range(3)]
+    _check(lib().ug_index_map_sizes(ctypes.byref(g), *[ctypes.byref(x) for x in n]),
+           "ug_index_map_sizes")
+    arrs = [np.zeros(x.value, dtype=np.int32) for x in n]
+    ptrs = [a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) for a in arrs]
+    _check(lib().ug_build_index_maps(ctypes.byref(g), *ptrs), "ug_build_index_maps")
+    return tuple(arrs)
+
+
+def visible_pairs(g: ug_geom):
+    """Per (batch, head): (hr_hr, hr_lr, lr_lr) visible query/key pairs."""
+    n = [ctypes.c_int64() for _ in range(3)]
+    _check(lib().ug_visible_pairs(ctypes.byref(g), *[ctypes.byref(x) for x in n]),
+           "ug_visible_pairs")
+    return tuple(x.value for x in n)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device tensor expected")
+    if not t.is_contiguous():
+        raise ValueError("contiguous tensor expected")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Plan:
+    """Owns a ug_plan (device index lists and RoPE tables) for one geometry."""
+
+    def __init__(self, **geom):
+        self.geom_kw = dict(geom)
+        self.g = make_geom(**geom)
+        h = ctypes.c_void_p()
+        _check(lib().ug_plan_create(ctypes.byref(self.g), ctypes.byref(h)), "ug_plan_create")
+        self.handle = h
+
+    def close(self):
+        if self.handle:
+            _check(lib().ug_plan_destroy(self.handle), "ug_plan_destroy")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            if getattr(self, "handle", None):
+                lib().ug_plan_destroy(self.handle)
+                self.handle = None
+        except Exception:
+            pass
+
+    # -- host-side views ---------------------------------------------------
+    def index_maps(self):
+        n = [ctypes.c_int64() for _ in range(3)]
+        _check(lib().ug_index_map_sizes(ctypes.byref(self.g), *[ctypes.byref(x) for x in n]),
+               "ug_index_map_sizes")
+        arrs = [np.zeros(x.value, dtype=np.int32) for x in n]
+        ptrs = [a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) for a in arrs]
+        _check(lib().ug_get_index_maps(self.handle, *ptrs), "ug_get_index_maps")
+        return tuple(arrs)
+
+    def workspace_bytes(self) -> int:
+        return int(lib().ug_layer_workspace_bytes(self.handle))
+
+    # -- the four steps --------------------------------------------------------
+    def permute_window_first(self, src, dst, stream=None) -> int:
+        return lib().ug_permute_window_first(self.handle, _ptr(src), _ptr(dst), _stream(stream))
+
+    def unpermute(self, src, dst, stream=None) -> int:
+        return lib().ug_unpermute(self.handle, _ptr(src), _ptr(dst), _stream(stream))
+
+    def rope_2d(self, x, y, token_set: int, stream=None) -> int:
+        return lib().ug_rope_2d(self.handle, _ptr(x), _ptr(y), int(token_set), _stream(stream))
+
+    def hier_local_attn_fwd(self, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse=None,
+                            stream=None) -> int:
+        return lib().ug_hier_local_attn_fwd(
+            self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr), _ptr(q_lr), _ptr(k_lr), _ptr(v_lr),
+            _ptr(o_hr), _ptr(o_lr), _ptr(lse), _stream(stream))
+
+    def layer_fwd(self, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, workspace,
+                  stream=None) -> int:
+        return lib().ug_layer_fwd(
+            self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr), _ptr(q_lr), _ptr(k_lr), _ptr(v_lr),
+            _ptr(o_hr), _ptr(o_lr), _ptr(lse), _ptr(workspace),
+            ctypes.c_int64(workspace.numel() * workspace.element_size()), _stream(stream))
+
+    def check_error(self, stream=None) -> int:
+        return lib().ug_check_error(self.handle, _stream(stream))
+
+
+# ---- convenience wrappers (allocate outputs with torch, raise on errors) -----
+
+def permute_window_first(plan: Plan, x: torch.Tensor) -> torch.Tensor:
+    out = torch.empty_like(x)
+    _check(plan.permute_window_first(x, out), "ug_permute_window_first")
+    return out
+
+
+def unpermute(plan: Plan, x: torch.Tensor) -> torch.Tensor:
+    out = torch.empty_like(x)
+    _check(plan.unpermute(x, out), "ug_unpermute")
+    return out
+
+
+def rope_2d(plan: Plan, x: torch.Tensor, token_set: int, inplace: bool = False) -> torch.Tensor:
+    out = x if inplace else torch.empty_like(x)
+    _check(plan.rope_2d(x, out, token_set), "ug_rope_2d")
+    return out
+
+
+def hier_local_attn_fwd(plan: Plan, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, want_lse=True):
+    o_hr = torch.empty_like(q_hr)
+    o_lr = torch.empty_like(q_lr) if q_lr is not None and q_lr.numel() else None
+    lse = None
+    if want_lse:
+        B, N, H, _ = q_hr.shape
+        L = q_lr.shape[1] if q_lr is not None else 0
+        lse = torch.empty((B, H, N + L), dtype=torch.float32, device=q_hr.device)
+    lr = (q_lr, k_lr, v_lr) if o_lr is not None else (None, None, None)
+    _check(plan.hier_local_attn_fwd(q_hr, k_hr, v_hr, *lr, o_hr, o_lr, lse),
+           "ug_hier_local_attn_fwd")
+    return o_hr, o_lr, lse
+
+
+def layer_forward(plan: Plan, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, workspace=None, want_lse=True):
+    """Whole layer on raster-order device tensors; returns (o_hr raster, o_lr, lse)."""
+    if workspace is None:
+        workspace = torch.empty(plan.workspace_bytes(), dtype=torch.uint8, device=q_hr.device)
+    o_hr = torch.empty_like(q_hr)
+    has_lr = q_lr is not None and q_lr.numel() > 0
+    o_lr = torch.empty_like(q_lr) if has_lr else None
+    lse = None
+    if want_lse:
+        B, N, H, _ = q_hr.shape
+        L = q_lr.shape[1] if has_lr else 0
+        lse = torch.empty((B, H, N + L), dtype=torch.float32, device=q_hr.device)
+    lr = (q_lr, k_lr, v_lr) if has_lr else (None, None, None)
+    _check(plan.layer_fwd(q_hr, k_hr, v_hr, *lr, o_hr, o_lr, lse, workspace), "ug_layer_fwd")
+    return o_hr, o_lr, lse

@@ -1,0 +1,205 @@
+/*
+ * ug.h -- C ABI of a B200 (sm_100a) library for one hierarchical-local-
+ * attention layer of UltraGen ("UltraGen: Efficient Ultra-High-Resolution
+ * Image Generation with Hierarchical Local Attention", arXiv 2510.16325).
+ *
+ * The layer, as the gist.science summaries of the paper state it
+ * (UltraGen-it, -fr, -es, -ar, -ko; sections cited per call below):
+ *   1. the high-res latent token grid is cut into fixed, non-overlapping
+ *      windows and its tokens are reordered window-first, so that each window
+ *      is one contiguous run of the sequence;
+ *   2. 2-D RoPE is applied; the positions of the low-res guidance tokens are
+ *      multiplied by rho (4 on the pages) to land on the high-res scale;
+ *   3. attention is block sparse: every high-res window attends to itself,
+ *      its neighbouring windows and all low-res tokens under one softmax; the
+ *      low-res tokens attend to each other only;
+ *   4. the high-res output is put back into raster order.
+ *
+ * Conventions shared by every call
+ *   - Tensors are bf16, contiguous, laid out [batch, tokens, heads, head_dim]
+ *     ("token-major"); the caller owns them.  Every device pointer must be
+ *     16-byte aligned (UG_ERR_ALIGNMENT otherwise).
+ *   - High-res tokens: N = grid_h * grid_w.  Raster order: token r sits at
+ *     row r / grid_w, column r % grid_w.  Window-first order: windows in
+ *     raster order (w = wy * (grid_w / win_w) + wx), each window's
+ *     T = win_h * win_w tokens in raster order inside it, so window w is the
+ *     range [w*T, (w+1)*T).
+ *   - Low-res tokens: L = lr_h * lr_w, raster order, never permuted.
+ *   - Launches are asynchronous on the given stream (a cudaStream_t passed as
+ *     a void*, NULL = the legacy default stream); nothing synchronises except
+ *     ug_check_error.  Only ug_plan_create allocates device memory and only
+ *     ug_plan_destroy frees it.
+ *   - Every call returns a ug_status; no C++ exception crosses the ABI.
+ *     Argument errors are reported before any work is queued.
+ */
+#ifndef UG_H_
+#define UG_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ug_status {
+  UG_OK = 0,
+  UG_ERR_INVALID_ARG = 1,  /* null pointer, bad geometry, bad token set         */
+  UG_ERR_UNSUPPORTED = 2,  /* a valid geometry this build does not run          */
+  UG_ERR_ALIGNMENT = 3,    /* a device pointer not 16-byte aligned              */
+  UG_ERR_ALIAS = 4,        /* output overlaps an input where that is not allowed */
+  UG_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed                 */
+  UG_ERR_TIMEOUT = 6,      /* a bounded device-side wait expired (kernel gave up) */
+  UG_ERR_NO_MEMORY = 7     /* host or device allocation failed in ug_plan_create */
+} ug_status;
+
+/* Token sets for ug_rope_2d: which grid the rows of x belong to and in which
+ * order, hence which RoPE positions they take. */
+typedef enum ug_token_set {
+  UG_HR_WINDOW_FIRST = 0, /* [B, N, h, d], high-res, window-first order */
+  UG_HR_RASTER = 1,       /* [B, N, h, d], high-res, raster order       */
+  UG_LR = 2               /* [B, L, h, d], low-res, raster order        */
+} ug_token_set;
+
+/* Problem statement (UltraGen-fr §2.A-B, UltraGen-ar §2.أ-ب): the token grid,
+ * the fixed window, the neighbourhood radius, the low-res grid and its RoPE
+ * scale rho, heads and head dim, the axial RoPE split. */
+typedef struct ug_geom {
+  int32_t batch;       /* B >= 1                                              */
+  int32_t grid_h;      /* high-res token grid H x W                           */
+  int32_t grid_w;
+  int32_t win_h;       /* window in tokens; must divide the grid exactly      */
+  int32_t win_w;
+  int32_t radius;      /* neighbourhood in windows, Chebyshev (1 -> 3x3)      */
+  int32_t lr_h;        /* low-res grid; 0 x 0 = no low-res tokens             */
+  int32_t lr_w;
+  double rho;          /* low-res RoPE position scale (4 on the pages), > 0   */
+  int32_t heads;       /* h >= 1                                              */
+  int32_t head_dim;    /* d; the attention runs d in {64, 128}                */
+  int32_t rope_dim_y;  /* channels [0, a_y) rotate with the row position      */
+  int32_t rope_dim_x;  /* channels [a_y, d) with the column; a_y + a_x = d,   */
+                       /* each a multiple of 8                                */
+  double rope_theta;   /* RoPE base, > 1 (10000)                               */
+  float softmax_scale; /* 0 -> 1/sqrt(head_dim)                               */
+} ug_geom;
+
+typedef struct ug_plan ug_plan; /* opaque: geometry, device index lists, RoPE
+                                   tables, device error word */
+
+/* ---- host-only helpers (no GPU needed) ---------------------------------- */
+
+/* Checks a geometry.  UG_OK, UG_ERR_INVALID_ARG (null, non-positive sizes,
+ * windows that do not tile the grid, a RoPE split that does not sum to d or
+ * has a segment not a multiple of 8, lr_h*lr_w == 0 with one of them != 0,
+ * rho <= 0, theta <= 1, negative radius, sizes whose element count passes
+ * 2^31 per tensor) or UG_ERR_UNSUPPORTED. */
+int ug_geom_validate(const ug_geom* g);
+
+/* Element counts of the three index maps of ug_build_index_maps. */
+int ug_index_map_sizes(const ug_geom* g, int64_t* n_perm, int64_t* n_nbr_off,
+                       int64_t* n_nbr_idx);
+
+/* Index maps, into caller-owned host arrays (sizes from ug_index_map_sizes):
+ *   perm[r]  (N entries): window-first position of raster token r
+ *            (UltraGen-fr §2.A "Ordre Window-First");
+ *   nbr_off  (nWin + 1) / nbr_idx: CSR lists, per window w (raster window
+ *            id), of the windows it attends to: Chebyshev distance <= radius,
+ *            clipped at the grid border, itself included, ascending
+ *            (UltraGen-ar §2.ب, attention mask, first item). */
+int ug_build_index_maps(const ug_geom* g, int32_t* perm, int32_t* nbr_off, int32_t* nbr_idx);
+
+/* Visible (query, key) pairs per (batch element, head): high-res query with
+ * high-res key, high-res query with low-res key, low-res with low-res.  The
+ * useful FLOPs of the attention are 4 * head_dim * heads * batch * (sum). */
+int ug_visible_pairs(const ug_geom* g, int64_t* hr_hr, int64_t* hr_lr, int64_t* lr_lr);
+
+const char* ug_status_string(int status);
+
+/* ---- plan ---------------------------------------------------------------- */
+
+/* Validates g, builds the index maps, the attention work lists and the RoPE
+ * tables on the host, allocates device memory for them and copies them once
+ * (synchronously) to the current CUDA device.  *out is NULL on failure. */
+int ug_plan_create(const ug_geom* g, ug_plan** out);
+int ug_plan_destroy(ug_plan* plan); /* NULL is allowed; synchronises the device */
+
+/* The plan's index maps, copied into caller-owned host arrays (as
+ * ug_build_index_maps).  Any of the three pointers may be NULL. */
+int ug_get_index_maps(const ug_plan* plan, int32_t* perm, int32_t* nbr_off, int32_t* nbr_idx);
+
+/* ---- the four steps of the layer (device pointers) ----------------------- */
+
+/* Step 1.  dst_wf[b, perm[r]] = src_raster[b, r] for every high-res token,
+ * whole [h, d] rows copied bit for bit.  src/dst: [B, N, h, d] bf16.
+ * UG_ERR_ALIAS if the two ranges overlap.
+ * (UltraGen-fr §2.A "Ordre Window-First"; UltraGen-es §2, window-first
+ * permutation bullet; UltraGen-ar §2.أ.) */
+int ug_permute_window_first(const ug_plan* plan, const void* src_raster, void* dst_wf,
+                            void* stream);
+
+/* Step 4.  dst_raster[b, r] = src_wf[b, perm[r]]; the inverse of step 1. */
+int ug_unpermute(const ug_plan* plan, const void* src_wf, void* dst_raster, void* stream);
+
+/* Step 2.  2-D axial RoPE of x into y (y == x allowed; any other overlap is
+ * UG_ERR_ALIAS).  x, y: [B, N, h, d] (high-res sets) or [B, L, h, d] (UG_LR).
+ * A high-res token at grid (row, col) takes positions (row, col); the low-res
+ * token (i, j) takes (rho*i, rho*j) (UltraGen-ar §2.ب "Scaled Positional
+ * Embeddings": the low-res position indices are multiplied by rho; UltraGen-fr
+ * §2.B).  Channels [0, a_y) rotate by pos_row * f_k, channels [a_y, d) by
+ * pos_col * f_k, f_k = theta^(-2k/a) for the k-th adjacent channel pair
+ * (2k, 2k+1) of the segment of a channels: (x0, x1) -> (x0 c - x1 s,
+ * x0 s + x1 c), c and s the fp32-rounded fp64 cos/sin of the angle.  Each
+ * output is formed from exact fp64 products, one fp64 add, and one
+ * round-to-nearest-even to bf16, so results are reproducible bit for bit.
+ * Applied to queries and keys, never to values. */
+int ug_rope_2d(const ug_plan* plan, const void* x, void* y, int token_set, void* stream);
+
+/* Step 3.  Block-sparse joint attention (UltraGen-ar §2.ب "Attention
+ * Masking"; UltraGen-es §2, guidance item; UltraGen-it §2, one softmax over a
+ * window's own tokens and the guidance).  Inputs (already rotated):
+ *   q_hr, k_hr, v_hr: [B, N, h, d], high-res, WINDOW-FIRST order;
+ *   q_lr, k_lr, v_lr: [B, L, h, d], low-res (ignored, may be NULL, if L = 0).
+ * A high-res query of window w sees the high-res keys of every window within
+ * Chebyshev distance radius of w and every low-res key; a low-res query sees
+ * the low-res keys only; scores are softmax_scale * <q, k>, one softmax per
+ * query over everything it sees, output = probabilities times values.
+ * Outputs: o_hr [B, N, h, d] (window-first), o_lr [B, L, h, d], bf16, fp32
+ * accumulation; lse (optional, NULL to skip): fp32 [B, h, N + L], natural
+ * log of the softmax denominator, high-res rows first (window-first order).
+ * The outputs may not overlap any input (UG_ERR_ALIAS).  Requires
+ * d in {64, 128} (UG_ERR_UNSUPPORTED).  A device-side wait that exceeds its
+ * bound makes the kernel give up and record UG_ERR_TIMEOUT, read by
+ * ug_check_error. */
+int ug_hier_local_attn_fwd(const ug_plan* plan, const void* q_hr, const void* k_hr,
+                           const void* v_hr, const void* q_lr, const void* k_lr,
+                           const void* v_lr, void* o_hr, void* o_lr, float* lse, void* stream);
+
+/* ---- the whole layer ------------------------------------------------------ */
+
+/* Bytes of device scratch that ug_layer_fwd needs (window-first copies of the
+ * high-res q, k, v and o, rotated low-res q and k), or -1 for a NULL plan. */
+int64_t ug_layer_workspace_bytes(const ug_plan* plan);
+
+/* Steps 1-4 in order on raster-order inputs: window-first permute of
+ * q_hr, k_hr, v_hr; RoPE of q and k (high-res at window-first positions,
+ * low-res at rho-scaled positions); attention; unpermute of the high-res
+ * output into o_hr (raster order).  q/k/v are not modified.  lse as in
+ * ug_hier_local_attn_fwd (its high-res rows stay in window-first order).
+ * workspace: caller-owned device scratch of at least
+ * ug_layer_workspace_bytes(plan) bytes, 256-byte aligned; the call uses it
+ * for intermediates only. */
+int ug_layer_fwd(const ug_plan* plan, const void* q_hr, const void* k_hr, const void* v_hr,
+                 const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr, void* o_lr,
+                 float* lse, void* workspace, int64_t workspace_bytes, void* stream);
+
+/* ---- errors ---------------------------------------------------------------- */
+
+/* Synchronises `stream`, then returns (and clears) the first status a kernel
+ * of this plan recorded on the device (UG_ERR_TIMEOUT), else UG_ERR_CUDA if
+ * the stream reports an error, else UG_OK. */
+int ug_check_error(const ug_plan* plan, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UG_H_ */
