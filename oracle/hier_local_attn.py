@@ -213,9 +213,10 @@ def rope_frequencies(a: int, theta: float) -> list:
 
 def _cos_sin_table(positions: Sequence[float], freqs: Sequence[float]):
     """fp32(cos(pos*f)), fp32(sin(pos*f)); angle = one fp64 product."""
+    shape = (len(positions), len(freqs))
     c = np.array([[math.cos(p * f) for f in freqs] for p in positions], dtype=np.float64)
     s = np.array([[math.sin(p * f) for f in freqs] for p in positions], dtype=np.float64)
-    return c.astype(np.float32), s.astype(np.float32)
+    return c.reshape(shape).astype(np.float32), s.reshape(shape).astype(np.float32)
 
 
 def rope_tables(g: Geometry) -> Dict[str, Tuple[np.ndarray, np.ndarray]]:

@@ -62,9 +62,21 @@ def sample_lr_tokens(g: O.Geometry, seed: int, n: int = 12) -> np.ndarray:
 
 
 def err_stats(got: np.ndarray, ref: np.ndarray, v_scale=None):
-    """(max-abs, mean-abs) of got - ref; [..., h, d] arrays.  With v_scale
-    ([h]) the error of each head is divided by that head's value scale."""
+    """(max-abs, mean-abs) of got - ref over [..., h, d] arrays.
+
+    Unit-variance inputs: the plain errors, held to MAX_ABS / MEAN_ABS.
+    Inputs with per-head scales (v_scale, shape [h]): the bound is stated for
+    unit variance, so each head's error is divided by its value scale; and
+    because larger q/k scales sharpen the softmax, outputs reach several
+    times the value scale, where the bf16 output format alone rounds by up to
+    half an ulp, at most 2^-8 |ref| (unit roundoff of an 8-bit significand).
+    That part is subtracted (never below zero)
+    before the max bound applies; the mean bound is unchanged.
+    """
     d = np.abs(got - ref)
-    if v_scale is not None:
-        d = d / np.asarray(v_scale, dtype=np.float64)[:, None]
-    return float(d.max()), float(d.mean())
+    if v_scale is None:
+        return float(d.max()), float(d.mean())
+    s = np.asarray(v_scale, dtype=np.float64)[:, None]
+    d = d / s
+    dmax = np.maximum(d - 2.0 ** -8 * np.abs(ref) / s, 0.0)
+    return float(dmax.max()), float(d.mean())
