@@ -35,8 +35,12 @@ EXPORTS = (
     "ug_geom_validate", "ug_index_map_sizes", "ug_build_index_maps", "ug_visible_pairs",
     "ug_status_string", "ug_plan_create", "ug_plan_destroy", "ug_get_index_maps",
     "ug_permute_window_first", "ug_unpermute", "ug_rope_2d", "ug_hier_local_attn_fwd",
-    "ug_layer_workspace_bytes", "ug_layer_fwd", "ug_check_error",
+    "ug_layer_workspace_bytes", "ug_layer_fwd", "ug_layer_fwd_static_scratch",
+    "ug_check_error",
 )
+
+# Capacity of the static scratch of ug_layer_fwd_static_scratch (ug.h).
+UG_STATIC_SCRATCH_BYTES = 32 << 20
 
 
 class UgError(RuntimeError):
@@ -87,6 +91,7 @@ def lib() -> ctypes.CDLL:
         "ug_hier_local_attn_fwd": (I32, [P, P, P, P, P, P, P, P, P, P, P]),
         "ug_layer_workspace_bytes": (I64, [P]),
         "ug_layer_fwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I64, P]),
+        "ug_layer_fwd_static_scratch": (I32, [P, P, P, P, P, P, P, P, P, P, P]),
         "ug_check_error": (I32, [P, P]),
     }
     for name, (res, args) in sig.items():
@@ -209,6 +214,14 @@ class Plan:
             self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr), _ptr(q_lr), _ptr(k_lr), _ptr(v_lr),
             _ptr(o_hr), _ptr(o_lr), _ptr(lse), _ptr(workspace),
             ctypes.c_int64(workspace.numel() * workspace.element_size()), _stream(stream))
+
+    def layer_fwd_static_scratch(self, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse,
+                                 stream=None) -> int:
+        """The layer without a caller workspace: its intermediates live in the
+        library's static device scratch (no device allocation on this call)."""
+        return lib().ug_layer_fwd_static_scratch(
+            self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr), _ptr(q_lr), _ptr(k_lr), _ptr(v_lr),
+            _ptr(o_hr), _ptr(o_lr), _ptr(lse), _stream(stream))
 
     def check_error(self, stream=None) -> int:
         return lib().ug_check_error(self.handle, _stream(stream))

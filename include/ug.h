@@ -191,6 +191,35 @@ int ug_layer_fwd(const ug_plan* plan, const void* q_hr, const void* k_hr, const 
                  const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr, void* o_lr,
                  float* lse, void* workspace, int64_t workspace_bytes, void* stream);
 
+/* Capacity in bytes of the static scratch of ug_layer_fwd_static_scratch. */
+#define UG_STATIC_SCRATCH_BYTES (32ll << 20)
+
+/* The paper has no counterpart to this call; it exists for callers that must
+ * not allocate device memory while they run the layer: servers that reserve
+ * device memory at start-up and forbid allocation while serving (cudaMalloc
+ * can synchronise the device and fragments a tuned pool), real-time
+ * pipelines with a fixed latency budget, hosts where another component owns
+ * all device memory.
+ * Same arguments and results as ug_layer_fwd without the workspace: the
+ * intermediates live in one static device array of UG_STATIC_SCRATCH_BYTES
+ * (32 MiB) that every GPU which loads this library holds until the process
+ * exits.  The call allocates nothing (no cudaMalloc/cudaFree, no allocating
+ * library routine); the plan is created beforehand, at set-up, by
+ * ug_plan_create (which does allocate).
+ *   - UG_ERR_UNSUPPORTED, before any work is queued, when the plan's
+ *     ug_layer_workspace_bytes exceeds UG_STATIC_SCRATCH_BYTES;
+ *     UG_ERR_INVALID_ARG when the plan's device is not the current device.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents.
+ *     Nothing in it needs clearing (each call writes what it reads), but calls
+ *     that overlap on the GPU race on it: issue them on one stream. */
+int ug_layer_fwd_static_scratch(const ug_plan* plan, const void* q_hr, const void* k_hr,
+                                const void* v_hr, const void* q_lr, const void* k_lr,
+                                const void* v_lr, void* o_hr, void* o_lr, float* lse,
+                                void* stream);
+
 /* ---- errors ---------------------------------------------------------------- */
 
 /* Synchronises `stream`, then returns (and clears) the first status a kernel

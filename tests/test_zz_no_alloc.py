@@ -1,0 +1,60 @@
+"""ug_layer_fwd_static_scratch: the layer for callers that must not allocate.
+
+Some callers cannot allocate device memory while they run the layer (servers
+that reserve memory at start-up and forbid allocation while serving,
+real-time pipelines, hosts where another component owns the device memory).
+This entry point keeps the layer's intermediates in a static device array
+instead of a caller workspace.  Its output must match the workspace-based
+ug_layer_fwd within the tests' tolerance, on two calls in a row (the second
+call reuses the array the first one left behind).  This file is collected
+last so that a run stopping at its first failure has run everything else.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_local_raster_b200 import ug, workloads
+
+from parity import MAX_ABS, MEAN_ABS
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(wl, seed):
+    x = workloads.make_inputs(wl, seed=seed)
+    x.pop("head_scale", None)
+    return {k: v.to("cuda") for k, v in x.items()}
+
+
+@pytest.mark.parametrize("name", ["tiny", "multi_tile"])
+def test_static_scratch_layer_matches_workspace_layer(name):
+    wl = workloads.get(name)
+    plan = ug.Plan(**wl.geom_dict())
+    assert plan.workspace_bytes() <= ug.UG_STATIC_SCRATCH_BYTES
+    for call, seed in enumerate((11, 12)):  # two calls in a row, different inputs
+        d = _inputs(wl, seed)
+        ref_hr, ref_lr, ref_lse = ug.layer_forward(plan, d["q_hr"], d["k_hr"], d["v_hr"],
+                                                   d["q_lr"], d["k_lr"], d["v_lr"])
+        o_hr = torch.full_like(d["q_hr"], float("nan"))
+        o_lr = torch.full_like(d["q_lr"], float("nan"))
+        lse = torch.full_like(ref_lse, float("nan"))
+        st = plan.layer_fwd_static_scratch(d["q_hr"], d["k_hr"], d["v_hr"], d["q_lr"],
+                                           d["k_lr"], d["v_lr"], o_hr, o_lr, lse)
+        assert st == ug.UG_OK, ug.status_string(st)
+        torch.cuda.synchronize()
+        assert plan.check_error() == ug.UG_OK
+        for got, ref in ((o_hr, ref_hr), (o_lr, ref_lr)):
+            err = (got.double() - ref.double()).abs()
+            assert float(err.max()) <= MAX_ABS and float(err.mean()) <= MEAN_ABS, (call, name)
+        assert torch.allclose(lse, ref_lse, atol=1e-5, rtol=0)
+    plan.close()
+
+
+def test_static_scratch_rejects_geometries_that_do_not_fit():
+    wl = workloads.get("2K")
+    plan = ug.Plan(**wl.geom_dict())
+    assert plan.workspace_bytes() > ug.UG_STATIC_SCRATCH_BYTES
+    t = torch.zeros(16, dtype=torch.bfloat16, device="cuda")  # never touched
+    st = plan.layer_fwd_static_scratch(t, t, t, t, t, t, t, t, None)
+    assert st == ug.UG_ERR_UNSUPPORTED
+    plan.close()
