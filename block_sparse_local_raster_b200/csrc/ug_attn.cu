@@ -16,16 +16,21 @@
 // CTA layout (320 threads):
 //   warps 0-3  softmax for query tile 0 (rows 0..127 of the CTA)
 //   warps 4-7  softmax for query tile 1 (rows 128..255)
-//   warp 8     TMA producer: Q once, then K_j, V_j into a 3-slot ring
+//   warp 8     TMA producer: Q once, then K_j, V_j into a 5-slot ring
 //   warp 9     TMEM allocation and the tcgen05.mma issuer
 // TMEM (512 columns x 128 lanes x 32 bit): S0 [0,128) S1 [128,256)
 //   O0 [256, 256+D) O1 [384, 384+D).  One TMEM lane = one query row, so the
-//   row max and row sum are in-thread (no shuffles needed).
-// Shared memory: Q0 Q1, K/V ring, P0 P1 (bf16 probabilities, K-major, 128-byte
-//   swizzle, the A operand of O += P V).
-// Pipeline per key block j (tiles ping-pong so that one softmax overlaps the
-//   other tile's MMAs):  S0=Q0 K_j^T, S1=Q1 K_j^T | softmax0(j) | O0+=P0 V_j,
-//   S0=Q0 K_{j+1}^T | softmax1(j) | O1+=P1 V_j, S1=Q1 K_{j+1}^T | ...
+//   row max and row sum are in-thread.  The softmax writes the bf16
+//   probabilities P_t over the first 64 columns of S_t, and O_t += P_t V_j
+//   reads its A operand straight from TMEM: P never touches shared memory,
+//   which leaves shared-memory bandwidth to the tensor pipe's Q, K and V reads
+//   and the TMA writes.
+// Pipeline: per key block j the MMA warp issues
+//   O0 += P0(j) V_j, S0(j+1) = Q0 K_{j+1}^T, O1 += P1(j) V_j, S1(j+1) = ...
+// so one tile's softmax runs while the tensor pipe works on the other tile;
+// the tensor pipe executes in issue order, so S_t(j+1) overwrites P_t(j) only
+// after O_t += P_t(j) V_j has read it, and the commit that signals S_t(j+1)
+// also covers that product (the softmax never waits for O separately).
 // Online softmax in the log2 domain with lazy rescaling: the running
 // reference max moves (and O, l are rescaled) only when a block's max exceeds
 // it by more than 8 (a factor 256), so probabilities stay <= 256 and O is
@@ -47,7 +52,7 @@ namespace ug {
 namespace {
 
 constexpr int kThreads = 320;
-constexpr int kStages = 3;
+constexpr int kStages = 5;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -56,11 +61,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 template <int D>
 struct Layout {
   static constexpr int kTileBytes = kRowsPerTile * D * 2;     // Q tile, K or V tile
-  static constexpr int kPBytes = kRowsPerTile * kKeysPerBlock * 2;
   static constexpr int kQ = 0;
   static constexpr int kKV = kQ + kTilesPerCta * kTileBytes;
-  static constexpr int kP = kKV + kStages * kTileBytes;
-  static constexpr int kBar = kP + kTilesPerCta * kPBytes;
+  static constexpr int kBar = kKV + kStages * kTileBytes;
   // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
   static constexpr int kNumBars = 1 + 2 * kStages + 3 * kTilesPerCta + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base (u32), abort flag (u32)
@@ -184,6 +187,17 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
+// D += A * B with A (M x K, K-major) read from TMEM columns starting at a_tmem.
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -203,21 +217,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
-  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
@@ -242,6 +241,21 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// 32 consecutive 32-bit TMEM columns of this thread's lane <- r[0..31].
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -253,6 +267,13 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// max of three fp32 values (sm_100 three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -356,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; r < kRegions; ++r)
           tma_load_4d(sbase + Lay::kQ + t * Lay::kTileBytes + r * kRowsPerTile * 128, mq, r * 64,
                       head, qt.q0 + t * kRowsPerTile, b, q_full);
+      // K_j then V_j, block after block: the order the MMA warp consumes them.
       int it = 0;
       bool ok = true;
       for (int j = 0; j < nblk && ok; ++j) {
@@ -400,16 +422,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                    kk > 0);
         }
       };
+      // O_t += P_t V: P_t (bf16, 128 x 128) sits in the first 64 columns of
+      // S_t, 16 keys per 8 columns; V (keys x D, D contiguous) is MN-major.
       auto issue_pv = [&](int t, int slot, bool acc) {
-        const uint32_t pa = sbase + Lay::kP + t * Lay::kPBytes;
         const uint32_t va = sbase + Lay::kKV + slot * Lay::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kKeysPerBlock / 16; ++kk) {
-          const uint32_t aoff = (kk / 4) * (kRowsPerTile * 128) + (kk % 4) * 32;
-          const uint32_t boff = kk * 16 * 128;
-          mma_bf16(tO[t], smem_desc(pa + aoff, 16, 1024),
-                   smem_desc(va + boff, kKeysPerBlock * 128, 1024), kIdO, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kKeysPerBlock / 16; ++kk)
+          mma_bf16_tmem_a(tO[t], tS[t] + kk * 8, smem_desc(va + kk * 16 * 128, kKeysPerBlock * 128, 1024),
+                          kIdO, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = wait1(q_full, 0);
       if (ok) ok = wait1(kv_full(0), 0);
@@ -424,12 +444,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < nblk && ok; ++j) {
         const int itv = 2 * j + 1, itk = 2 * j + 2;
         const int sv = itv % kStages, sk = itk % kStages;
+        const bool more = j + 1 < nblk;
         if (!(ok = wait1(kv_full(sv), (uint32_t)(itv / kStages) & 1u))) break;
         if (!(ok = wait1(p_full(0), (uint32_t)j & 1u))) break;
         fence_after();
         issue_pv(0, sv, j > 0);
-        mma_commit(o_done(0));
-        const bool more = j + 1 < nblk;
+        if (!more) mma_commit(o_done(0));
         if (more) {
           if (!(ok = wait1(kv_full(sk), (uint32_t)(itk / kStages) & 1u))) break;
           fence_after();
@@ -439,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait1(p_full(1), (uint32_t)j & 1u))) break;
         fence_after();
         issue_pv(1, sv, j > 0);
-        mma_commit(o_done(1));
+        if (!more) mma_commit(o_done(1));
         mma_commit(kv_empty(sv));
         if (more) {
           issue_s(1, sk);
@@ -458,7 +478,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + (t ? 128u : 0u);
     const uint32_t tO = tmem + lane_base + 256u + (t ? 128u : 0u);
-    uint8_t* p_row = smem + Lay::kP + t * Lay::kPBytes + row * 128;
     const int tok = qt.q0 + t * kRowsPerTile + row;  // query token in its tensor
     const int q_w = tok / P.T;
     const int q_wy = q_w / P.nwx, q_wx = q_w - (q_w / P.nwx) * P.nwx;
@@ -467,6 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < nblk; ++j) {
       const uint32_t e = P.kvlist[qt.list_off + j];
+      // S_t(j) complete; the commit that signals it also covers every earlier
+      // MMA of this CTA, in particular O_t += P_t(j-1) V_{j-1}.
       if (!(ok = wait_warp(s_full(t), (uint32_t)j & 1u))) break;
       fence_after();
       float s[kKeysPerBlock];
@@ -497,58 +518,60 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      float mx = s[0];
+      // Row max: four independent chains of three-input maxima.
+      float mc[4];
 #pragma unroll
-      for (int i = 1; i < kKeysPerBlock; ++i) mx = fmaxf(mx, s[i]);
+      for (int c = 0; c < 4; ++c) mc[c] = fmaxf(s[2 * c], s[2 * c + 1]);
+#pragma unroll
+      for (int i = 8; i < kKeysPerBlock; i += 8) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mc[c] = fmax3(mc[c], s[i + 2 * c], s[i + 2 * c + 1]);
+      }
+      const float mx = fmax3(fmaxf(mc[0], mc[1]), mc[2], mc[3]);
       const float m_blk = mx * P.scale_log2;
       const bool rescale = m_blk > m_ref + kRescaleThreshold;
       const float m_new = rescale ? m_blk : m_ref;
       const float alpha = rescale ? fast_exp2(m_ref - m_new) : 1.0f;
       const float m_use = m_new == kNegInf ? 0.0f : m_new;
       m_ref = m_new;
-      if (j > 0) {
-        // O += P V of the previous block must be complete before its P
-        // buffer is overwritten and before O is rescaled.  It was issued
-        // ahead of this block's S, so it has normally retired already.
-        if (!(ok = wait_warp(o_done(t), (uint32_t)(j - 1) & 1u))) break;
-        fence_after();
-        if (__any_sync(0xFFFFFFFFu, rescale)) {
+      if (j > 0 && __any_sync(0xFFFFFFFFu, rescale)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 16; ++c) {
-            float o[16];
-            tmem_ld16(tO + c * 16, o);
-            tmem_ld_wait();
+        for (int c = 0; c < D / 16; ++c) {
+          float o[16];
+          tmem_ld16(tO + c * 16, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] *= alpha;
-            tmem_st16(tO + c * 16, o);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 16; ++i) o[i] *= alpha;
+          tmem_st16(tO + c * 16, o);
         }
       }
-      // p = 2^(s*scale*log2e - m): row sum in fp32, P row to shared memory
-      // as bf16, K-major with the 128-byte swizzle (16-byte chunk c of a
-      // 128-byte row lands at chunk c ^ (row % 8)).
-      float rowsum = 0.0f;
+      // p = 2^(s*scale*log2e - m): fp32 row sum; bf16 pairs (even key in the
+      // low half) over the first 64 columns of S_t, the A operand of O += P V.
+      const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
+      const float2 nm2 = make_float2(-m_use, -m_use);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < kKeysPerBlock / 8; ++c) {
-        float p[8];
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          p[i] = fast_exp2(fmaf(s[8 * c + i], P.scale_log2, -m_use));
-          rowsum += p[i];
+        for (int i = 0; i < 64; i += 2) {
+          const int k = 64 * h + i;
+          const float2 x = __ffma2_rn(make_float2(s[k], s[k + 1]), sc2, nm2);
+          const float2 pp = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          acc[(i / 2) & 3] = __fadd2_rn(acc[(i / 2) & 3], pp);
+          pk[i / 2] = pack_bf16(pp.x, pp.y);
         }
-        const uint4 v = make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
-                                   pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
-        const int region = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(p_row + region * (kRowsPerTile * 128) + ((cc ^ (row & 7)) << 4)) = v;
+        tmem_st32u(tS + 32 * h, pk);
       }
-      l = l * alpha + rowsum;
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const float2 a4 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+      l = l * alpha + (a4.x + a4.y);
+      tmem_st_wait();
       fence_before();
       mbar_arrive(p_full(t));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = wait_warp(o_done(t), (uint32_t)(nblk - 1) & 1u);
+    if (ok) ok = wait_warp(o_done(t), 0);
     if (ok) {
       fence_after();
       const int ntok = qt.lowres ? P.L : P.N;
