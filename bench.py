@@ -2,9 +2,9 @@
 """Benchmark of one hierarchical-local-attention layer on B200.
 
 A step is one pass of the whole layer over one batch of synthetic raster-order
-inputs already resident in HBM: window-first permute of q, k, v (3 launches),
-RoPE of q and k, high-res and low-res (4), block-sparse attention (1),
-unpermute of the output (1).  The metric is useful attention TFLOP/s
+inputs already resident in HBM: window-first permute of q, k, v with the RoPE
+of q and k applied in the same pass (3 launches), RoPE of the low-res q and k
+(2), block-sparse attention (1), unpermute of the output (1).  The metric is useful attention TFLOP/s
 (4 * head_dim FLOPs per visible query-key pair per head) over the step, with
 ms per layer; the attention kernel alone is also timed and set against the
 measured bf16 tensor peak.
@@ -274,11 +274,9 @@ def run_ug(args, wl, world, rank, local):
             raise ug.UgError(st, what)
 
     def step(ev=None):
-        chk(plan.permute_window_first(d["q_hr"], ws_q), "permute q")
-        chk(plan.permute_window_first(d["k_hr"], ws_k), "permute k")
+        chk(plan.permute_rope_window_first(d["q_hr"], ws_q), "permute+rope q")
+        chk(plan.permute_rope_window_first(d["k_hr"], ws_k), "permute+rope k")
         chk(plan.permute_window_first(d["v_hr"], ws_v), "permute v")
-        chk(plan.rope_2d(ws_q, ws_q, ug.UG_HR_WINDOW_FIRST), "rope q")
-        chk(plan.rope_2d(ws_k, ws_k, ug.UG_HR_WINDOW_FIRST), "rope k")
         if L:
             chk(plan.rope_2d(d["q_lr"], ws_ql, ug.UG_LR), "rope q_lr")
             chk(plan.rope_2d(d["k_lr"], ws_kl, ug.UG_LR), "rope k_lr")
@@ -290,7 +288,7 @@ def run_ug(args, wl, world, rank, local):
             ev[1].record(stream)
         chk(plan.unpermute(ws_o, o_hr), "unpermute")
 
-    launches_per_step = 3 + 2 + (2 if L else 0) + 1 + 1
+    launches_per_step = 3 + (2 if L else 0) + 1 + 1
     flops = useful_flops(wl)
 
     for _ in range(args.warmup):

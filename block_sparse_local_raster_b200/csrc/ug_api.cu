@@ -104,12 +104,13 @@ int ug_plan_create(const ug_geom* g, ug_plan** out) {
     build_neighbours(*g, p->nbr_off, p->nbr_idx);
     build_attention_lists(*g, p->nbr_off, p->nbr_idx, p->qtiles, p->kvlist, &p->n_hr_ctas,
                           &p->n_lr_ctas);
-    std::vector<float> tables;
-    build_rope_tables(*g, p->rope, tables);
+    std::vector<float> tables32;
+    build_rope_tables(*g, p->rope, tables32);
+    const std::vector<double> tables(tables32.begin(), tables32.end());
     // One device block: [err (256 B)] [rope tables] [qtiles] [kvlist]
     const size_t a_err = 0;
     const size_t a_rope = 256;
-    const size_t a_qt = (a_rope + tables.size() * sizeof(float) + 255) / 256 * 256;
+    const size_t a_qt = (a_rope + tables.size() * sizeof(double) + 255) / 256 * 256;
     const size_t a_kv = (a_qt + p->qtiles.size() * sizeof(QTile) + 255) / 256 * 256;
     const size_t total = a_kv + std::max<size_t>(1, p->kvlist.size()) * sizeof(uint32_t);
     if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return UG_ERR_CUDA; }
@@ -120,11 +121,11 @@ int ug_plan_create(const ug_geom* g, ug_plan** out) {
     }
     char* base = static_cast<char*>(p->d_mem);
     p->d_err = reinterpret_cast<int*>(base + a_err);
-    p->d_rope = reinterpret_cast<float*>(base + a_rope);
+    p->d_rope = reinterpret_cast<double*>(base + a_rope);
     p->d_qtiles = reinterpret_cast<QTile*>(base + a_qt);
     p->d_kvlist = reinterpret_cast<uint32_t*>(base + a_kv);
     std::vector<char> host(total, 0);
-    std::memcpy(host.data() + a_rope, tables.data(), tables.size() * sizeof(float));
+    std::memcpy(host.data() + a_rope, tables.data(), tables.size() * sizeof(double));
     std::memcpy(host.data() + a_qt, p->qtiles.data(), p->qtiles.size() * sizeof(QTile));
     std::memcpy(host.data() + a_kv, p->kvlist.data(), p->kvlist.size() * sizeof(uint32_t));
     if (cudaMemcpy(p->d_mem, host.data(), total, cudaMemcpyHostToDevice) != cudaSuccess) {
@@ -170,6 +171,15 @@ static int permute_common(const ug_plan* p, const void* src, void* dst, bool inv
 
 int ug_permute_window_first(const ug_plan* p, const void* src_raster, void* dst_wf, void* s) {
   return permute_common(p, src_raster, dst_wf, false, s);
+}
+
+int ug_permute_rope_window_first(const ug_plan* p, const void* src_raster, void* dst_wf,
+                                 void* s) {
+  if (!p || !src_raster || !dst_wf) return UG_ERR_INVALID_ARG;
+  if (!aligned16(src_raster) || !aligned16(dst_wf)) return UG_ERR_ALIGNMENT;
+  const int64_t n = hr_bytes(p);
+  if (overlap(src_raster, n, dst_wf, n)) return UG_ERR_ALIAS;
+  return launch_permute_rope(p, src_raster, dst_wf, as_stream(s));
 }
 
 int ug_unpermute(const ug_plan* p, const void* src_wf, void* dst_raster, void* s) {
@@ -245,11 +255,9 @@ int ug_layer_fwd(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   if (overlap(workspace, ws, o_hr, nh) || overlap(workspace, ws, o_lr, nl))
     return UG_ERR_ALIAS;
   int st;
-  if ((st = ug_permute_window_first(p, q_hr, q_wf, s)) != UG_OK) return st;
-  if ((st = ug_permute_window_first(p, k_hr, k_wf, s)) != UG_OK) return st;
+  if ((st = ug_permute_rope_window_first(p, q_hr, q_wf, s)) != UG_OK) return st;
+  if ((st = ug_permute_rope_window_first(p, k_hr, k_wf, s)) != UG_OK) return st;
   if ((st = ug_permute_window_first(p, v_hr, v_wf, s)) != UG_OK) return st;
-  if ((st = ug_rope_2d(p, q_wf, q_wf, UG_HR_WINDOW_FIRST, s)) != UG_OK) return st;
-  if ((st = ug_rope_2d(p, k_wf, k_wf, UG_HR_WINDOW_FIRST, s)) != UG_OK) return st;
   if (p->L > 0) {
     if ((st = ug_rope_2d(p, q_lr, q_lr_r, UG_LR, s)) != UG_OK) return st;
     if ((st = ug_rope_2d(p, k_lr, k_lr_r, UG_LR, s)) != UG_OK) return st;

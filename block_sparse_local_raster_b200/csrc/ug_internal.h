@@ -35,8 +35,10 @@ constexpr uint32_t kBlockIndexMask = (1u << 29) - 1;
 constexpr uint32_t kBlockLowres = 1u << 29;
 constexpr uint32_t kBlockMasked = 1u << 30;
 
-// Offsets (in floats) of the RoPE tables inside the plan's table buffer.
-// Each table is [coordinate][pair k], fp32; cos and sin separately.
+// Offsets (in elements) of the RoPE tables inside the plan's table buffer.
+// Each table is [coordinate][pair k]; cos and sin separately.  The values
+// are the fp32-rounded cos/sin, held in fp64 (exactly) so that the kernels
+// need no conversion to form exact fp64 products.
 struct RopeTables {
   int64_t hr_y_cos, hr_y_sin, hr_x_cos, hr_x_sin;
   int64_t lr_y_cos, lr_y_sin, lr_x_cos, lr_x_sin;
@@ -62,7 +64,7 @@ struct ug_plan {
   ug::RopeTables rope;
 
   void* d_mem;             // one device allocation holding everything below
-  float* d_rope;           // RoPE tables
+  double* d_rope;          // RoPE tables
   ug::QTile* d_qtiles;     // attention query CTAs
   uint32_t* d_kvlist;      // attention key-block lists
   int* d_err;              // first device-side error status (0 = none)
@@ -83,6 +85,7 @@ void build_rope_tables(const ug_geom& g, RopeTables& off, std::vector<float>& da
 // Kernel launchers (one .cu each).  Arguments are already checked.
 int launch_permute(const ug_plan* p, const void* src, void* dst, bool inverse, cudaStream_t s);
 int launch_rope(const ug_plan* p, const void* x, void* y, int token_set, cudaStream_t s);
+int launch_permute_rope(const ug_plan* p, const void* src, void* dst, cudaStream_t s);
 int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                      const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
                      void* o_lr, float* lse, cudaStream_t s);

@@ -34,7 +34,8 @@ UG_LR = 2
 EXPORTS = (
     "ug_geom_validate", "ug_index_map_sizes", "ug_build_index_maps", "ug_visible_pairs",
     "ug_status_string", "ug_plan_create", "ug_plan_destroy", "ug_get_index_maps",
-    "ug_permute_window_first", "ug_unpermute", "ug_rope_2d", "ug_hier_local_attn_fwd",
+    "ug_permute_window_first", "ug_permute_rope_window_first", "ug_unpermute", "ug_rope_2d",
+    "ug_hier_local_attn_fwd",
     "ug_layer_workspace_bytes", "ug_layer_fwd", "ug_layer_fwd_static_scratch",
     "ug_check_error",
 )
@@ -86,6 +87,7 @@ def lib() -> ctypes.CDLL:
         "ug_plan_destroy": (I32, [P]),
         "ug_get_index_maps": (I32, [P, pi32, pi32, pi32]),
         "ug_permute_window_first": (I32, [P, P, P, P]),
+        "ug_permute_rope_window_first": (I32, [P, P, P, P]),
         "ug_unpermute": (I32, [P, P, P, P]),
         "ug_rope_2d": (I32, [P, P, P, I32, P]),
         "ug_hier_local_attn_fwd": (I32, [P, P, P, P, P, P, P, P, P, P, P]),
@@ -196,6 +198,10 @@ class Plan:
     def permute_window_first(self, src, dst, stream=None) -> int:
         return lib().ug_permute_window_first(self.handle, _ptr(src), _ptr(dst), _stream(stream))
 
+    def permute_rope_window_first(self, src, dst, stream=None) -> int:
+        return lib().ug_permute_rope_window_first(self.handle, _ptr(src), _ptr(dst),
+                                                  _stream(stream))
+
     def unpermute(self, src, dst, stream=None) -> int:
         return lib().ug_unpermute(self.handle, _ptr(src), _ptr(dst), _stream(stream))
 
@@ -232,6 +238,12 @@ class Plan:
 def permute_window_first(plan: Plan, x: torch.Tensor) -> torch.Tensor:
     out = torch.empty_like(x)
     _check(plan.permute_window_first(x, out), "ug_permute_window_first")
+    return out
+
+
+def permute_rope_window_first(plan: Plan, x: torch.Tensor) -> torch.Tensor:
+    out = torch.empty_like(x)
+    _check(plan.permute_rope_window_first(x, out), "ug_permute_rope_window_first")
     return out
 
 

@@ -136,6 +136,16 @@ int ug_get_index_maps(const ug_plan* plan, int32_t* perm, int32_t* nbr_off, int3
 int ug_permute_window_first(const ug_plan* plan, const void* src_raster, void* dst_wf,
                             void* stream);
 
+/* Steps 1 and 2 in one pass: dst_wf[b, perm[r]] = RoPE(src_raster[b, r]) at
+ * the token's grid position, for high-res queries and keys.  Bit for bit the
+ * same as ug_permute_window_first followed by ug_rope_2d(UG_HR_WINDOW_FIRST)
+ * (the rotation depends only on the token's position), with one read and one
+ * write of the tensor instead of two each.  src/dst: [B, N, h, d] bf16;
+ * UG_ERR_ALIAS if they overlap.  (UltraGen-fr §2.A "Ordre Window-First" and
+ * §2.B; UltraGen-ar §2.ب "Scaled Positional Embeddings".) */
+int ug_permute_rope_window_first(const ug_plan* plan, const void* src_raster, void* dst_wf,
+                                 void* stream);
+
 /* Step 4.  dst_raster[b, r] = src_wf[b, perm[r]]; the inverse of step 1. */
 int ug_unpermute(const ug_plan* plan, const void* src_wf, void* dst_raster, void* stream);
 
@@ -180,9 +190,10 @@ int ug_hier_local_attn_fwd(const ug_plan* plan, const void* q_hr, const void* k_
 int64_t ug_layer_workspace_bytes(const ug_plan* plan);
 
 /* Steps 1-4 in order on raster-order inputs: window-first permute of
- * q_hr, k_hr, v_hr; RoPE of q and k (high-res at window-first positions,
- * low-res at rho-scaled positions); attention; unpermute of the high-res
- * output into o_hr (raster order).  q/k/v are not modified.  lse as in
+ * q_hr, k_hr, v_hr (q and k with their RoPE applied in the same pass, as
+ * ug_permute_rope_window_first); RoPE of the low-res q and k (rho-scaled
+ * positions); attention; unpermute of the high-res output into o_hr (raster
+ * order).  q/k/v are not modified.  lse as in
  * ug_hier_local_attn_fwd (its high-res rows stay in window-first order).
  * workspace: caller-owned device scratch of at least
  * ug_layer_workspace_bytes(plan) bytes, 256-byte aligned; the call uses it

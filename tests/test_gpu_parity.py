@@ -89,6 +89,26 @@ def test_rope_bit_exact(name):
     assert p.check_error() == ug.UG_OK
 
 
+@pytest.mark.parametrize("name", SMALL + BIG)
+def test_permute_rope_fused_bit_exact(name):
+    """Window-first permute with RoPE in the same pass equals the oracle's
+    rotation at window-first positions of the permuted tensor."""
+    wl = workloads.get(name)
+    g = ogeom(wl)
+    p = plan(wl)
+    tab = O.rope_tables(g)
+    x = rand((wl.batch, wl.n_hr, wl.heads, wl.head_dim), 250)
+    y = ug.permute_rope_window_first(p, x.to(DEV))
+    torch.cuda.synchronize()
+    assert p.check_error() == ug.UG_OK
+    yb, xb = bits(y), bits(x)
+    heads = list(range(wl.heads)) if name != "8K" else [0, 11, 23]
+    for h in heads:
+        want = O.rope_2d(O.permute_window_first(xb[:, :, h:h + 1], g), g, O.HR_WINDOW_FIRST,
+                         tables=tab)
+        np.testing.assert_array_equal(yb[:, :, h:h + 1], want, err_msg=f"{name} head {h}")
+
+
 # ----------------------------------------------------------------- attention alone
 
 def attn_inputs(wl, seed):
@@ -239,6 +259,8 @@ def test_error_statuses_on_device_pointers():
     mis = flat[1:1 + x.numel()].view_as(x)  # 2-byte offset
     assert p.permute_window_first(mis, out) == ug.UG_ERR_ALIGNMENT
     assert p.permute_window_first(x, x) == ug.UG_ERR_ALIAS
+    assert p.permute_rope_window_first(x, x) == ug.UG_ERR_ALIAS
+    assert p.permute_rope_window_first(mis, out) == ug.UG_ERR_ALIGNMENT
     assert p.unpermute(x, x) == ug.UG_ERR_ALIAS
     assert p.rope_2d(x, x, 7) == ug.UG_ERR_INVALID_ARG
     assert p.rope_2d(x, x, ug.UG_HR_RASTER) == ug.UG_OK  # exact in place is allowed
