@@ -268,6 +268,12 @@ int ug_layer_fwd(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   return ug_unpermute(p, o_wf, o_hr, s);
 }
 
+int ug_plan_set_wait_timeout(ug_plan* p, int64_t ns) {
+  if (!p || ns <= 0) return UG_ERR_INVALID_ARG;
+  p->wait_timeout_ns = ns;
+  return UG_OK;
+}
+
 int ug_check_error(const ug_plan* p, void* s) {
   if (!p) return UG_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(as_stream(s)) != cudaSuccess) return UG_ERR_CUDA;

@@ -314,8 +314,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto wait1 = [&](uint32_t bar, uint32_t par) {
     return mbar_wait(bar, par, abort, err, timeout_ns, false);
   };
+  // Draining (loads and MMAs already in flight) always gets the full bound,
+  // whatever the plan's wait limit: TMEM and shared memory are released only
+  // after the asynchronous units are done with them.
   auto drain_wait = [&](uint32_t bar, uint32_t par) {
-    return mbar_wait(bar, par, abort, err, timeout_ns, true);
+    return mbar_wait(bar, par, abort, err, kDefaultWaitTimeoutNs, true);
   };
   auto wait_warp = [&](uint32_t bar, uint32_t par) {
     return __all_sync(0xFFFFFFFFu, mbar_wait(bar, par, abort, err, timeout_ns, false)) != 0;

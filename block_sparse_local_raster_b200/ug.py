@@ -37,7 +37,7 @@ EXPORTS = (
     "ug_permute_window_first", "ug_permute_rope_window_first", "ug_unpermute", "ug_rope_2d",
     "ug_hier_local_attn_fwd",
     "ug_layer_workspace_bytes", "ug_layer_fwd", "ug_layer_fwd_static_scratch",
-    "ug_check_error",
+    "ug_plan_set_wait_timeout", "ug_check_error",
 )
 
 # Capacity of the static scratch of ug_layer_fwd_static_scratch (ug.h).
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
         "ug_layer_workspace_bytes": (I64, [P]),
         "ug_layer_fwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I64, P]),
         "ug_layer_fwd_static_scratch": (I32, [P, P, P, P, P, P, P, P, P, P, P]),
+        "ug_plan_set_wait_timeout": (I32, [P, I64]),
         "ug_check_error": (I32, [P, P]),
     }
     for name, (res, args) in sig.items():
@@ -228,6 +229,9 @@ class Plan:
         return lib().ug_layer_fwd_static_scratch(
             self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr), _ptr(q_lr), _ptr(k_lr), _ptr(v_lr),
             _ptr(o_hr), _ptr(o_lr), _ptr(lse), _stream(stream))
+
+    def set_wait_timeout(self, ns: int) -> int:
+        return lib().ug_plan_set_wait_timeout(self.handle, ctypes.c_int64(int(ns)))
 
     def check_error(self, stream=None) -> int:
         return lib().ug_check_error(self.handle, _stream(stream))

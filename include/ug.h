@@ -233,6 +233,14 @@ int ug_layer_fwd_static_scratch(const ug_plan* plan, const void* q_hr, const voi
 
 /* ---- errors ---------------------------------------------------------------- */
 
+/* Bound, in ns, on each device-side wait of this plan's attention kernel
+ * (default 2e9).  A wait that exceeds it makes the kernel record
+ * UG_ERR_TIMEOUT, stop issuing work, let its in-flight loads and MMAs finish,
+ * free its tensor memory and exit; later CTAs of the launch skip their work.
+ * A very small bound makes ordinary waits expire, which exercises that path
+ * without any fault.  UG_ERR_INVALID_ARG for a NULL plan or ns <= 0. */
+int ug_plan_set_wait_timeout(ug_plan* plan, int64_t ns);
+
 /* Synchronises `stream`, then returns (and clears) the first status a kernel
  * of this plan recorded on the device (UG_ERR_TIMEOUT), else UG_ERR_CUDA if
  * the stream reports an error, else UG_OK. */
