@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="4K", choices=list(workloads.CONFIGS))
+    ap.add_argument("--config", default="4K", choices=list(workloads.CONFIGS) + list(workloads.EXTRA_CONFIGS))
     ap.add_argument("--impl", default="ug", choices=["ug", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=12)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -457,7 +457,7 @@ def main():
     world, rank, local = dist_env()
     if args.gpus != world and world > 1:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
-    wl = workloads.CONFIGS[args.config]
+    wl = workloads.get(args.config)
     if args.impl == "reference":
         run_reference(args, wl, world, rank)
         return

@@ -62,7 +62,7 @@ int ug_visible_pairs(const ug_geom* g, int64_t* hr_hr, int64_t* hr_lr, int64_t* 
   std::vector<int32_t> off, idx;
   build_neighbours(*g, off, idx);
   const int64_t T = (int64_t)g->win_h * g->win_w;
-  const int64_t N = (int64_t)g->grid_h * g->grid_w, L = (int64_t)g->lr_h * g->lr_w;
+  const int64_t N = (int64_t)g->grid_h * g->grid_w, L = global_tokens(*g);
   if (hr_hr) *hr_hr = (int64_t)idx.size() * T * T;
   if (hr_lr) *hr_lr = N * L;
   if (lr_lr) *lr_lr = L * L;
@@ -92,7 +92,7 @@ int ug_plan_create(const ug_geom* g, ug_plan** out) {
   if (!p) return UG_ERR_NO_MEMORY;
   p->g = *g;
   p->N = (int64_t)g->grid_h * g->grid_w;
-  p->L = (int64_t)g->lr_h * g->lr_w;
+  p->L = global_tokens(*g);
   p->T = (int64_t)g->win_h * g->win_w;
   p->nwy = g->grid_h / g->win_h;
   p->nwx = g->grid_w / g->win_w;

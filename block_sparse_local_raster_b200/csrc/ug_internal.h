@@ -45,6 +45,11 @@ struct RopeTables {
   int64_t total;
 };
 
+// Tokens of the global set: text tokens, then the low-res grid.
+inline int64_t global_tokens(const ug_geom& g) {
+  return (int64_t)g.text_len + (int64_t)g.lr_h * g.lr_w;
+}
+
 // Upper bound of a device-side wait before a kernel gives up (ns).
 constexpr int64_t kDefaultWaitTimeoutNs = 2000000000ll;
 
@@ -52,7 +57,7 @@ constexpr int64_t kDefaultWaitTimeoutNs = 2000000000ll;
 
 struct ug_plan {
   ug_geom g;
-  int64_t N, L, T;   // high-res tokens, low-res tokens, tokens per window
+  int64_t N, L, T;   // high-res tokens, global (text + low-res) tokens, tokens per window
   int32_t nwy, nwx;  // windows per axis
   float scale;       // softmax scale actually used
   int device;

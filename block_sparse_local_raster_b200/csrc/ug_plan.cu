@@ -13,7 +13,8 @@ namespace ug {
 int validate(const ug_geom* g) {
   if (!g) return UG_ERR_INVALID_ARG;
   if (g->batch < 1 || g->grid_h < 1 || g->grid_w < 1 || g->win_h < 1 || g->win_w < 1 ||
-      g->heads < 1 || g->head_dim < 2 || g->radius < 0 || g->lr_h < 0 || g->lr_w < 0)
+      g->heads < 1 || g->head_dim < 2 || g->radius < 0 || g->lr_h < 0 || g->lr_w < 0 ||
+      g->text_len < 0)
     return UG_ERR_INVALID_ARG;
   // Fixed non-overlapping windows that tile the grid; no padding.
   if (g->grid_h % g->win_h || g->grid_w % g->win_w) return UG_ERR_INVALID_ARG;
@@ -25,7 +26,7 @@ int validate(const ug_geom* g) {
     return UG_ERR_INVALID_ARG;
   const int64_t row = (int64_t)g->heads * g->head_dim;
   const int64_t n = (int64_t)g->grid_h * g->grid_w;
-  const int64_t l = (int64_t)g->lr_h * g->lr_w;
+  const int64_t l = global_tokens(*g);
   if (row * 2 % 16) return UG_ERR_UNSUPPORTED;
   if ((int64_t)g->batch * n * row >= (1ll << 31) || (int64_t)g->batch * l * row >= (1ll << 31))
     return UG_ERR_INVALID_ARG;
@@ -59,13 +60,14 @@ void build_neighbours(const ug_geom& g, std::vector<int32_t>& off, std::vector<i
 }
 
 // Per query CTA (256 rows), the 128-key blocks holding at least one key that
-// some row of the CTA may see.  A block is "full" when every valid row of the
+// some row of the CTA may see.  The global tokens (text, then low-res) form
+// one key set that every query sees.  A block is "full" when every valid row of the
 // CTA sees every key of the block (then the kernel skips per-pair tests).
 void build_attention_lists(const ug_geom& g, const std::vector<int32_t>& nbr_off,
                            const std::vector<int32_t>& nbr_idx, std::vector<QTile>& qtiles,
                            std::vector<uint32_t>& kvlist, int32_t* n_hr_ctas,
                            int32_t* n_lr_ctas) {
-  const int64_t N = (int64_t)g.grid_h * g.grid_w, L = (int64_t)g.lr_h * g.lr_w;
+  const int64_t N = (int64_t)g.grid_h * g.grid_w, L = global_tokens(g);
   const int64_t T = (int64_t)g.win_h * g.win_w;
   const int nwx = g.grid_w / g.win_w;
   const int64_t BK = kKeysPerBlock;

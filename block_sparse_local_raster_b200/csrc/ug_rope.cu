@@ -89,6 +89,7 @@ struct RopeArgs {
   int32_t my, mx;      // a_y / 2, a_x / 2
   int32_t set;         // ug_token_set
   int32_t grid_w, win_h, win_w, nwx, T, lr_w;
+  int32_t text_len;    // UG_LR: leading text rows, copied unrotated
 };
 
 // One warp per token row: lanes walk the row's 16-byte chunks (coalesced);
@@ -103,8 +104,14 @@ __global__ void __launch_bounds__(kThreads) rope_kernel(const RopeArgs a) {
     const int32_t t = (int32_t)(row % a.n_tok);
     int32_t pr, pc;  // grid row / column of the token
     if (a.set == UG_LR) {
-      pr = t / a.lr_w;
-      pc = t - pr * a.lr_w;
+      if (t < a.text_len) {  // text token: no grid position, no rotation
+        const uint4* __restrict__ xs = a.x + row * a.row_chunks;
+        uint4* __restrict__ ys = a.y + row * a.row_chunks;
+        for (int32_t c = lane; c < a.row_chunks; c += 32) ys[c] = xs[c];
+        continue;
+      }
+      pr = (t - a.text_len) / a.lr_w;
+      pc = (t - a.text_len) - pr * a.lr_w;
     } else if (a.set == UG_HR_RASTER) {
       pr = t / a.grid_w;
       pc = t - pr * a.grid_w;
@@ -204,6 +211,7 @@ int launch_rope(const ug_plan* p, const void* x, void* y, int set, cudaStream_t 
   a.nwx = p->nwx;
   a.T = (int32_t)p->T;
   a.lr_w = p->g.lr_w;
+  a.text_len = p->g.text_len;
   if (a.n_rows == 0) return UG_OK;
   const int blocks = grid_for(p, (a.n_rows + (kThreads / 32) - 1) / (kThreads / 32));
   if (a.head_chunks == 16)

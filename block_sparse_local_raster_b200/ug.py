@@ -58,6 +58,7 @@ class ug_geom(ctypes.Structure):
         ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("rope_dim_y", ctypes.c_int32), ("rope_dim_x", ctypes.c_int32),
         ("rope_theta", ctypes.c_double), ("softmax_scale", ctypes.c_float),
+        ("text_len", ctypes.c_int32),
     ]
 
 

@@ -12,7 +12,9 @@ i.i.d. normal draws, rounded once to bf16.
 
 Draw recipe (every config): ``torch.Generator('cpu').manual_seed(seed)``, then
 ``randn`` in the order q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, each shaped
-``[batch, tokens, heads, head_dim]`` in raster token order, fp32.  Configs with
+``[batch, tokens, heads, head_dim]`` in raster token order, fp32.  The ``_lr``
+tensors hold the global tokens: ``text_len`` text tokens first (drawn like the
+rest; no text encoder is involved), then the low-res grid.  Configs with
 ``head_scale`` then draw one U[0.5, 2] factor per (tensor in q, k, v; head),
 shared by the high-res and low-res parts and by every batch element, and
 multiply it in fp32.  Finally every tensor is rounded to bf16 (round to nearest
@@ -45,6 +47,7 @@ class Workload:
     rope_theta: float = 10000.0
     softmax_scale: float = 0.0  # 0 -> 1/sqrt(head_dim)
     head_scale: bool = False  # per-(tensor, head) U[0.5, 2] factor
+    text_len: int = 0  # text tokens at the head of the global tensors
 
     @property
     def n_hr(self) -> int:
@@ -52,7 +55,8 @@ class Workload:
 
     @property
     def n_lr(self) -> int:
-        return self.lr_h * self.lr_w
+        """Rows of the global (``_lr``) tensors: text tokens, then low-res."""
+        return self.text_len + self.lr_h * self.lr_w
 
     @property
     def window_tokens(self) -> int:
@@ -65,7 +69,7 @@ class Workload:
                     lr_h=self.lr_h, lr_w=self.lr_w, rho=self.rho, heads=self.heads,
                     head_dim=self.head_dim, rope_dim_y=self.rope_dim_y,
                     rope_dim_x=self.rope_dim_x, rope_theta=self.rope_theta,
-                    softmax_scale=self.softmax_scale)
+                    softmax_scale=self.softmax_scale, text_len=self.text_len)
 
 
 def _wl(name, batch, grid, win, lr, heads, d, split, radius=1, rho=4.0, **kw) -> Workload:
@@ -85,6 +89,13 @@ CONFIGS: Dict[str, Workload] = {
                   head_scale=True),
 }
 
+# The 4K layer with the text tokens of the joint MMDiT sequence added to the
+# global set (512: the T5 prompt length of FLUX-class models).
+EXTRA_CONFIGS: Dict[str, Workload] = {
+    "4K-text": _wl("4K-text", 1, (256, 256), (16, 16), (64, 64), 24, 128, (64, 64),
+                   text_len=512),
+}
+
 # Small geometries for element-by-element parity: several tiles, ragged tails,
 # non-square grids, windows that do not divide the 128-token tile, radius 0/2,
 # no low-res set, one window covering the whole grid.
@@ -99,12 +110,17 @@ TEST_GEOMETRIES: Dict[str, Workload] = {
     "asym_split": _wl("asym_split", 1, (32, 64), (16, 16), (4, 8), 2, 128, (32, 96),
                       rho=8.0),
     "rho_frac": _wl("rho_frac", 1, (32, 32), (8, 8), (6, 6), 1, 64, (32, 32), rho=2.5),
+    "text77": _wl("text77", 1, (48, 32), (16, 16), (6, 4), 2, 128, (64, 64), text_len=77),
+    "text_only": _wl("text_only", 1, (32, 24), (8, 8), (0, 0), 2, 64, (32, 32),
+                     text_len=130),
 }
 
 
 def get(name: str) -> Workload:
     if name in CONFIGS:
         return CONFIGS[name]
+    if name in EXTRA_CONFIGS:
+        return EXTRA_CONFIGS[name]
     return TEST_GEOMETRIES[name]
 
 

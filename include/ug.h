@@ -24,7 +24,13 @@
  *     raster order (w = wy * (grid_w / win_w) + wx), each window's
  *     T = win_h * win_w tokens in raster order inside it, so window w is the
  *     range [w*T, (w+1)*T).
- *   - Low-res tokens: L = lr_h * lr_w, raster order, never permuted.
+ *   - Global tokens: the tensors named *_lr hold L = text_len + lr_h * lr_w
+ *     rows: the text tokens first (the MMDiT joint sequence concatenates
+ *     text, high-res and low-res tokens: UltraGen-it §2, LoRA item;
+ *     UltraGen-fr §2.C), then the low-res guidance grid in raster order.
+ *     They are never permuted.  Text tokens are seen by every query and see
+ *     the global tokens only, exactly like the low-res tokens; they carry no
+ *     grid position, so RoPE leaves them unchanged.
  *   - Launches are asynchronous on the given stream (a cudaStream_t passed as
  *     a void*, NULL = the legacy default stream); nothing synchronises except
  *     ug_check_error.  Only ug_plan_create allocates device memory and only
@@ -80,6 +86,7 @@ typedef struct ug_geom {
                        /* each a multiple of 8                                */
   double rope_theta;   /* RoPE base, > 1 (10000)                               */
   float softmax_scale; /* 0 -> 1/sqrt(head_dim)                               */
+  int32_t text_len;    /* text tokens at the head of the global tensors, >= 0 */
 } ug_geom;
 
 typedef struct ug_plan ug_plan; /* opaque: geometry, device index lists, RoPE
@@ -90,7 +97,7 @@ typedef struct ug_plan ug_plan; /* opaque: geometry, device index lists, RoPE
 /* Checks a geometry.  UG_OK, UG_ERR_INVALID_ARG (null, non-positive sizes,
  * windows that do not tile the grid, a RoPE split that does not sum to d or
  * has a segment not a multiple of 8, lr_h*lr_w == 0 with one of them != 0,
- * rho <= 0, theta <= 1, negative radius, sizes whose element count passes
+ * rho <= 0, theta <= 1, negative radius or text_len, sizes whose element count passes
  * 2^31 per tensor) or UG_ERR_UNSUPPORTED. */
 int ug_geom_validate(const ug_geom* g);
 
@@ -108,7 +115,8 @@ int ug_index_map_sizes(const ug_geom* g, int64_t* n_perm, int64_t* n_nbr_off,
 int ug_build_index_maps(const ug_geom* g, int32_t* perm, int32_t* nbr_off, int32_t* nbr_idx);
 
 /* Visible (query, key) pairs per (batch element, head): high-res query with
- * high-res key, high-res query with low-res key, low-res with low-res.  The
+ * high-res key, high-res query with global key, global with global (global =
+ * text and low-res tokens, L = text_len + lr_h * lr_w of them).  The
  * useful FLOPs of the attention are 4 * head_dim * heads * batch * (sum). */
 int ug_visible_pairs(const ug_geom* g, int64_t* hr_hr, int64_t* hr_lr, int64_t* lr_lr);
 
@@ -150,7 +158,8 @@ int ug_permute_rope_window_first(const ug_plan* plan, const void* src_raster, vo
 int ug_unpermute(const ug_plan* plan, const void* src_wf, void* dst_raster, void* stream);
 
 /* Step 2.  2-D axial RoPE of x into y (y == x allowed; any other overlap is
- * UG_ERR_ALIAS).  x, y: [B, N, h, d] (high-res sets) or [B, L, h, d] (UG_LR).
+ * UG_ERR_ALIAS).  x, y: [B, N, h, d] (high-res sets) or [B, L, h, d] (UG_LR,
+ * the global tokens: rows [0, text_len) are text and are copied unchanged).
  * A high-res token at grid (row, col) takes positions (row, col); the low-res
  * token (i, j) takes (rho*i, rho*j) (UltraGen-ar §2.ب "Scaled Positional
  * Embeddings": the low-res position indices are multiplied by rho; UltraGen-fr
@@ -167,10 +176,12 @@ int ug_rope_2d(const ug_plan* plan, const void* x, void* y, int token_set, void*
  * Masking"; UltraGen-es §2, guidance item; UltraGen-it §2, one softmax over a
  * window's own tokens and the guidance).  Inputs (already rotated):
  *   q_hr, k_hr, v_hr: [B, N, h, d], high-res, WINDOW-FIRST order;
- *   q_lr, k_lr, v_lr: [B, L, h, d], low-res (ignored, may be NULL, if L = 0).
+ *   q_lr, k_lr, v_lr: [B, L, h, d], global tokens, text then low-res
+ *                     (ignored, may be NULL, if L = 0).
  * A high-res query of window w sees the high-res keys of every window within
- * Chebyshev distance radius of w and every low-res key; a low-res query sees
- * the low-res keys only; scores are softmax_scale * <q, k>, one softmax per
+ * Chebyshev distance radius of w and every global key; a global (text or
+ * low-res) query sees the global keys only; scores are softmax_scale * <q, k>,
+ * one softmax per
  * query over everything it sees, output = probabilities times values.
  * Outputs: o_hr [B, N, h, d] (window-first), o_lr [B, L, h, d], bf16, fp32
  * accumulation; lse (optional, NULL to skip): fp32 [B, h, N + L], natural
@@ -186,13 +197,13 @@ int ug_hier_local_attn_fwd(const ug_plan* plan, const void* q_hr, const void* k_
 /* ---- the whole layer ------------------------------------------------------ */
 
 /* Bytes of device scratch that ug_layer_fwd needs (window-first copies of the
- * high-res q, k, v and o, rotated low-res q and k), or -1 for a NULL plan. */
+ * high-res q, k, v and o, rotated global q and k), or -1 for a NULL plan. */
 int64_t ug_layer_workspace_bytes(const ug_plan* plan);
 
 /* Steps 1-4 in order on raster-order inputs: window-first permute of
  * q_hr, k_hr, v_hr (q and k with their RoPE applied in the same pass, as
- * ug_permute_rope_window_first); RoPE of the low-res q and k (rho-scaled
- * positions); attention; unpermute of the high-res output into o_hr (raster
+ * ug_permute_rope_window_first); RoPE of the global q and k (rho-scaled
+ * low-res positions, text rows unchanged); attention; unpermute of the high-res output into o_hr (raster
  * order).  q/k/v are not modified.  lse as in
  * ug_hier_local_attn_fwd (its high-res rows stay in window-first order).
  * workspace: caller-owned device scratch of at least

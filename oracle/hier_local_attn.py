@@ -19,6 +19,8 @@ Local Attention") in language xx; the section follows.
   * Low-res guidance tokens with RoPE positions multiplied by rho (= 4 on the
     pages) (UltraGen-ar §2.ب "Scaled Positional Embeddings";
     UltraGen-fr §2.B; UltraGen-es §2 "Guía Global de Baja Resolución").
+  * The joint MMDiT sequence concatenates text, high-res and low-res tokens
+    (UltraGen-it §2, LoRA item; UltraGen-fr §2.C).
   * The attention mask: a high-res window sees itself, its adjacent windows and
     every low-res token; low-res tokens see each other
     (UltraGen-ar §2.ب "Attention Masking"; UltraGen-es §2, last bullet of the
@@ -36,7 +38,10 @@ Readings where the pages are silent (each is listed in the design notes):
     cos/sin evaluated in fp64 by the C library and rounded to fp32; each output
     is x0*c - x1*s (or x0*s + x1*c) from exact fp64 products with one fp64
     rounding, then rounded to nearest-even bf16;
-  * low-res queries do not see high-res keys; softmax scale 1/sqrt(d).
+  * low-res queries do not see high-res keys; softmax scale 1/sqrt(d);
+  * text tokens (the pages give no mask for them) join the low-res tokens in
+    one global set, placed first: every query sees them, they see the global
+    set only, and having no grid position they are not rotated.
 
 bf16 values travel as their uint16 bit patterns (numpy has no bf16 type).
 """
@@ -70,6 +75,7 @@ class Geometry:
     rope_dim_x: int
     rope_theta: float = 10000.0
     softmax_scale: float = 0.0
+    text_len: int = 0
 
     @staticmethod
     def from_dict(d: dict) -> "Geometry":
@@ -83,6 +89,8 @@ class Geometry:
             raise ValueError("axial RoPE split must sum to head_dim")
         if self.rope_dim_y % 2 or self.rope_dim_x % 2:
             raise ValueError("RoPE segments must hold whole pairs")
+        if self.text_len < 0:
+            raise ValueError("text_len must be >= 0")
 
     @property
     def N(self) -> int:
@@ -90,7 +98,8 @@ class Geometry:
 
     @property
     def L(self) -> int:
-        return self.lr_h * self.lr_w
+        """Global tokens: ``text_len`` text tokens, then the low-res grid."""
+        return self.text_len + self.lr_h * self.lr_w
 
     @property
     def T(self) -> int:
@@ -236,10 +245,16 @@ def rope_tables(g: Geometry) -> Dict[str, Tuple[np.ndarray, np.ndarray]]:
 
 
 def token_coords(g: Geometry, token_set: str, tokens: Optional[np.ndarray] = None):
-    """(row, col) grid coordinates of each token of a token set."""
+    """(row, col) grid coordinates of each token of a token set.
+
+    For the global set (LOWRES) the index counts the text tokens first; a text
+    token has no grid position and gets (-1, -1).
+    """
     if token_set == LOWRES:
         t = np.arange(g.L, dtype=np.int64) if tokens is None else np.asarray(tokens, np.int64)
-        return np.divmod(t, g.lr_w)
+        lr = t - g.text_len
+        row, col = np.divmod(np.maximum(lr, 0), max(g.lr_w, 1))
+        return np.where(lr < 0, -1, row), np.where(lr < 0, -1, col)
     t = np.arange(g.N, dtype=np.int64) if tokens is None else np.asarray(tokens, np.int64)
     if token_set == HR_WINDOW_FIRST:
         t = raster_index(g)[t]
@@ -267,14 +282,19 @@ def rope_2d_f64(x64: np.ndarray, g: Geometry, token_set: str,
     """RoPE in fp64 before the final rounding.  x64: [B, T, h, d]."""
     tab = rope_tables(g) if tables is None else tables
     row, col = token_coords(g, token_set, tokens)
+    text = row < 0  # text tokens: no position, left as they are
+    out = x64.copy()
+    if text.all():
+        return out
+    row, col, keep = row[~text], col[~text], np.nonzero(~text)[0]
     ky, kx = ("lr_y", "lr_x") if token_set == LOWRES else ("hr_y", "hr_x")
     cy, sy = tab[ky][0][row], tab[ky][1][row]  # [T, a_y/2]
     cx, sx = tab[kx][0][col], tab[kx][1][col]
     ay = g.rope_dim_y
-    out = np.empty_like(x64)
     c64 = lambda v: v.astype(np.float64)[None, :, None, :]
-    out[..., :ay] = rope_rotate_f64(x64[..., :ay], c64(cy), c64(sy))
-    out[..., ay:] = rope_rotate_f64(x64[..., ay:], c64(cx), c64(sx))
+    x = x64[:, keep]
+    out[:, keep, :, :ay] = rope_rotate_f64(x[..., :ay], c64(cy), c64(sy))
+    out[:, keep, :, ay:] = rope_rotate_f64(x[..., ay:], c64(cx), c64(sx))
     return out
 
 
@@ -301,7 +321,7 @@ def visibility(g: Geometry, hr_order: str, rows: np.ndarray) -> np.ndarray:
 
     Rows and keys index the joint sequence (high-res first, in ``hr_order``).
     High-res query: high-res key in a window at Chebyshev distance <= radius,
-    or any low-res key.  Low-res query: low-res keys only.
+    or any global (text or low-res) key.  Global query: global keys only.
     """
     N, L = g.N, g.L
     wy, wx = window_coords_of_tokens(g, hr_order)

@@ -58,6 +58,8 @@ def sample_lr_tokens(g: O.Geometry, seed: int, n: int = 12) -> np.ndarray:
         return np.zeros(0, dtype=np.int64)
     rng = np.random.default_rng(seed + 1)
     t = {0, g.L - 1} | set(rng.integers(0, g.L, size=n).tolist())
+    if g.text_len:  # both sides of the text / low-res boundary
+        t |= {g.text_len - 1, min(g.text_len, g.L - 1)}
     return np.array(sorted(t), dtype=np.int64)
 
 

@@ -36,7 +36,8 @@ def g_of(wl, **over):
     return ug.make_geom(**d)
 
 
-ALL = list(workloads.CONFIGS.values()) + list(workloads.TEST_GEOMETRIES.values())
+ALL = (list(workloads.CONFIGS.values()) + list(workloads.EXTRA_CONFIGS.values())
+       + list(workloads.TEST_GEOMETRIES.values()))
 
 
 @pytest.mark.parametrize("wl", ALL, ids=lambda w: w.name)
@@ -73,6 +74,13 @@ def test_useful_flops_of_the_benchmark_configs():
         assert 4 * wl.head_dim * pairs * wl.heads * wl.batch == want[name], name
 
 
+def test_useful_flops_with_text_tokens():
+    """4K with 512 text tokens: G = 512 + 64^2 = 4608 global tokens, so
+    256^2 * 14^2 ... = 138,674,176 + 65,536 * 4608 + 4608^2 pairs per head."""
+    wl = workloads.EXTRA_CONFIGS["4K-text"]
+    assert ug.visible_pairs(g_of(wl)) == (138_674_176, 301_989_888, 21_233_664)
+
+
 @pytest.mark.parametrize("over,status", [
     (dict(win_h=7), ug.UG_ERR_INVALID_ARG),            # windows must tile the grid
     (dict(grid_w=0), ug.UG_ERR_INVALID_ARG),
@@ -86,6 +94,9 @@ def test_useful_flops_of_the_benchmark_configs():
     (dict(heads=1 << 20), ug.UG_ERR_INVALID_ARG),       # element count past 2^31
     (dict(), ug.UG_OK),
     (dict(lr_h=0, lr_w=0), ug.UG_OK),
+    (dict(text_len=-1), ug.UG_ERR_INVALID_ARG),
+    (dict(text_len=77), ug.UG_OK),
+    (dict(lr_h=0, lr_w=0, text_len=5), ug.UG_OK),      # text as the only global tokens
 ])
 def test_geometry_validation(over, status):
     assert ug.geom_validate(g_of(workloads.CONFIGS["tiny"], **over)) == status

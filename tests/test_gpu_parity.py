@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 SMALL = list(workloads.TEST_GEOMETRIES) + ["tiny"]
-BIG = ["2K", "4K", "8K", "4K-CFG"]
+BIG = ["2K", "4K", "8K", "4K-CFG", "4K-text"]
 
 
 def rand(shape, seed):
@@ -236,6 +236,26 @@ def test_window_output_ignores_keys_outside_its_neighbourhood():
     s = slice(w * g.T, (w + 1) * g.T)
     assert torch.equal(o_hr[:, s], o2_hr[:, s])
     assert torch.equal(o_lr, o2_lr)
+
+
+def test_global_rows_ignore_high_res_inputs():
+    """Text and low-res queries see only the global set: replacing every
+    high-res q/k/v leaves their outputs bit-identical, and changing the text
+    keys changes the high-res outputs (every query sees the text tokens)."""
+    wl = workloads.get("text77")
+    p = plan(wl)
+    x = attn_inputs(wl, 510)
+    o_hr, o_lr, _ = run_attn(p, x)
+    y = dict(x)
+    for k in ("q_hr", "k_hr", "v_hr"):
+        y[k] = -x[k]
+    _, o2_lr, _ = run_attn(p, y)
+    assert torch.equal(o_lr, o2_lr)
+    z = dict(x)
+    z["v_lr"] = x["v_lr"].clone()
+    z["v_lr"][:, :wl.text_len] = 4.0
+    o3_hr, _, _ = run_attn(p, z)
+    assert ((o3_hr.float() - o_hr.float()).abs() > 0).float().mean() > 0.99
 
 
 def test_constant_values_give_constant_output():
