@@ -440,3 +440,147 @@ def visible_pairs(g: Geometry, block_rows: int = 512) -> Dict[str, int]:
         cnt["lr_lr"] += int(v[~hr][:, N:].sum())
         assert not v[~hr][:, :N].any()
     return cnt
+
+
+# --------------------------------------------------------------------------
+# Backward pass.  The gradients of the layer's loss with respect to q, k, v,
+# given dO, the gradient with respect to its output.  The pages train LoRA
+# adapters on the q/k/v projections of the low-res guidance
+# (UltraGen-ar §2.ج, UltraGen-fr §2.C), which needs these gradients through
+# the attention and the RoPE.  Written from the derivative of
+# O = softmax(scale * Q K^T, masked) V, row by row:
+#   dV = P^T dO;  dP = dO V^T;  dS = P * (dP - rowsum(P * dP));
+#   dQ = scale * dS K;  dK = scale * dS^T Q.
+# RoPE is a rotation per channel pair, so its backward is the transposed
+# rotation: (g0, g1) -> (g0 c + g1 s, -g0 s + g1 c), with the same fp32 c, s.
+# --------------------------------------------------------------------------
+
+def _as_f64(a: np.ndarray) -> np.ndarray:
+    """uint16 arrays hold bf16 patterns; float64 arrays are taken as they are."""
+    return a if a.dtype == np.float64 else bf16_to_f64(a)
+
+
+def attention_backward_rows(Q, K, V, dO, vis, scale):
+    """One chunk of query rows, fp64.  Q, dO: [r, d]; K, V: [n, d];
+    vis: [r, n].  Returns (dQ [r, d], dK part [n, d], dV part [n, d]): the
+    rows' own dQ and their contributions to every key's dK and dV."""
+    s = (Q @ K.T) * scale
+    s[~vis] = -np.inf
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    p /= p.sum(axis=1, keepdims=True)
+    dP = dO @ V.T
+    D = (p * dP).sum(axis=1, keepdims=True)
+    dS = p * (dP - D)
+    return scale * (dS @ K), scale * (dS.T @ Q), p.T @ dO
+
+
+def rows_seeing(g: Geometry, hr_order: str, keys: np.ndarray, block_rows: int = 1024):
+    """Every query row (joint sequence) that sees at least one of ``keys``."""
+    keys = np.asarray(keys, dtype=np.int64)
+    if (keys >= g.N).any():
+        return np.arange(g.N + g.L, dtype=np.int64)  # every query sees a global key
+    out = []
+    for i0 in range(0, g.N + g.L, block_rows):
+        r = np.arange(i0, min(g.N + g.L, i0 + block_rows))
+        out.append(r[visibility(g, hr_order, r)[:, keys].any(axis=1)])
+    return np.concatenate(out) if out else np.zeros(0, dtype=np.int64)
+
+
+def attention_backward(q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, do_hr, do_lr, g: Geometry,
+                       hr_order: str, rows: Optional[np.ndarray] = None,
+                       keys: Optional[np.ndarray] = None,
+                       heads: Optional[Iterable[int]] = None, chunk_elems: int = 1 << 24):
+    """Gradients of the joint attention on bf16 inputs (uint16 patterns; fp64
+    arrays are also accepted and used as they are).
+
+    q..v and do: as ``attention`` ([B, N, h, d] high-res in ``hr_order``,
+    [B, L, h, d] global).  rows: query rows whose dQ is wanted; keys: key
+    rows whose dK, dV are wanted (joint-sequence indices; default all).
+    Returns dQ [B, len(rows), h, d], dK and dV [B, len(keys), h, d], fp64.
+    """
+    N, L = g.N, g.L
+    n = N + L
+    rows = np.arange(n, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    keys = np.arange(n, dtype=np.int64) if keys is None else np.asarray(keys, np.int64)
+    heads = list(range(g.heads)) if heads is None else list(heads)
+    need = np.union1d(rows, rows_seeing(g, hr_order, keys)) if keys.size else rows
+    where_row = {int(r): i for i, r in enumerate(rows)}
+    B = q_hr.shape[0]
+    dQ = np.zeros((B, rows.size, g.heads, g.head_dim))
+    dK = np.zeros((B, keys.size, g.heads, g.head_dim))
+    dV = np.zeros((B, keys.size, g.heads, g.head_dim))
+    step = max(1, chunk_elems // max(1, n))
+    for b in range(B):
+        for h in heads:
+            joint = lambda a, c: np.concatenate([_as_f64(a[b, :, h]), _as_f64(c[b, :, h])])
+            Q, K, V, dO = joint(q_hr, q_lr), joint(k_hr, k_lr), joint(v_hr, v_lr), joint(do_hr, do_lr)
+            for i0 in range(0, need.size, step):
+                r = need[i0:i0 + step]
+                dq, dk, dv = attention_backward_rows(Q[r], K, V, dO[r],
+                                                     visibility(g, hr_order, r), g.scale)
+                dK[b, :, h] += dk[keys]
+                dV[b, :, h] += dv[keys]
+                for j, ri in enumerate(r):
+                    i = where_row.get(int(ri))
+                    if i is not None:
+                        dQ[b, i, h] = dq[j]
+    return dQ, dK, dV
+
+
+def rope_2d_backward_f64(g64: np.ndarray, g: Geometry, token_set: str,
+                         tokens: Optional[np.ndarray] = None, tables=None) -> np.ndarray:
+    """Gradient through RoPE: each channel pair's rotation transposed, i.e.
+    (g0, g1) -> (g0 c + g1 s, -g0 s + g1 c) with the forward's fp32 c, s
+    (products exact in fp64, one fp64 rounding each).  Text rows pass."""
+    tab = rope_tables(g) if tables is None else tables
+    neg = {k: (c, -s) for k, (c, s) in tab.items()}  # R(-a) = R(a)^T: c kept, s negated
+    return rope_2d_f64(g64, g, token_set, tokens, neg)
+
+
+def rope_2d_backward(g_bits: np.ndarray, g: Geometry, token_set: str,
+                     tokens: Optional[np.ndarray] = None, tables=None) -> np.ndarray:
+    """bf16 in, bf16 out (round to nearest even), as ``rope_2d``."""
+    return f64_to_bf16(rope_2d_backward_f64(bf16_to_f64(g_bits), g, token_set, tokens, tables))
+
+
+def layer_backward(inp: Dict[str, np.ndarray], dout: Dict[str, np.ndarray], g: Geometry,
+                   rows: Optional[np.ndarray] = None, keys: Optional[np.ndarray] = None,
+                   heads: Optional[Iterable[int]] = None, exact_rope: bool = False):
+    """Gradients of the whole layer on raster-order inputs.
+
+    inp: uint16 q/k/v as ``layer_forward``; dout: uint16 do_hr [B, N, h, d]
+    (raster) and do_lr [B, L, h, d].  The forward's bf16 rounding of the
+    rotated q and k passes gradients unchanged.  rows: joint rows (raster
+    high-res first) whose dq is wanted; keys: joint rows whose dk, dv are
+    wanted.  Returns fp64 (dq, dk, dv), gradients w.r.t. the unrotated inputs.
+    exact_rope: keep the rotated q and k in fp64 (no bf16 rounding), the
+    layer in exact arithmetic.
+    """
+    tab = rope_tables(g)
+    N, L = g.N, g.L
+    rows = np.arange(N + L, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    keys = np.arange(N + L, dtype=np.int64) if keys is None else np.asarray(keys, np.int64)
+    heads = list(range(g.heads)) if heads is None else list(heads)
+    B = inp["q_hr"].shape[0]
+    dq = np.zeros((B, rows.size, g.heads, g.head_dim))
+    dk = np.zeros((B, keys.size, g.heads, g.head_dim))
+    dv = np.zeros((B, keys.size, g.heads, g.head_dim))
+    g1 = dataclasses.replace(g, heads=1)
+    for h in heads:
+        sl = slice(h, h + 1)
+        rot = ((lambda a, s: rope_2d_f64(bf16_to_f64(a), g, s, tables=tab)) if exact_rope
+               else (lambda a, s: rope_2d(a, g, s, tables=tab)))
+        q = (rot(inp["q_hr"][:, :, sl], HR_RASTER), rot(inp["q_lr"][:, :, sl], LOWRES))
+        k = (rot(inp["k_hr"][:, :, sl], HR_RASTER), rot(inp["k_lr"][:, :, sl], LOWRES))
+        a, kk, vv = attention_backward(q[0], k[0], inp["v_hr"][:, :, sl], q[1], k[1],
+                                       inp["v_lr"][:, :, sl], dout["do_hr"][:, :, sl],
+                                       dout["do_lr"][:, :, sl], g1, HR_RASTER, rows, keys)
+        for src, idx, dst in ((a, rows, dq), (kk, keys, dk)):
+            hr, lr = idx < N, idx >= N
+            if hr.any():
+                dst[:, hr, h] = rope_2d_backward_f64(src[:, hr], g, HR_RASTER, idx[hr], tab)[:, :, 0]
+            if lr.any():
+                dst[:, lr, h] = rope_2d_backward_f64(src[:, lr], g, LOWRES, idx[lr] - N, tab)[:, :, 0]
+        dv[:, :, h] = vv[:, :, 0]
+    return dq, dk, dv
