@@ -10,6 +10,8 @@ ms per layer; the attention kernel alone is also timed and set against the
 measured bf16 tensor peak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4K] [--impl ug|reference]
+  python bench.py --op warm_start [--config 4K|8K]   (the warm-start kernel alone)
+  python bench.py --op backward [--config 4K]        (the layer's backward pass)
 
 N > 1 runs under torchrun, one rank per GPU; every rank runs its own layer on
 its own inputs (independent problems, weak scaling, no data-path collective);
@@ -51,6 +53,7 @@ def parse():
     ap.add_argument("--impl", default="ug", choices=["ug", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=12)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="layer", choices=["layer", "warm_start", "backward"])
     return ap.parse_args()
 
 
@@ -452,11 +455,251 @@ def run_ug(args, wl, world, rank, local):
         dist.destroy_process_group()
 
 
+def run_backward(args, wl, world, rank, local):
+    """The layer's backward pass: gradients w.r.t. the raster q, k, v given
+    the forward's outputs and lse.  A step recomputes the window-first
+    rotated operands (5 permutes, 2 of them with RoPE; RoPE of the global q,
+    k), runs the attention backward (D, dQ, dK/dV kernels; timed alone with
+    events) and maps dq, dk back with the transposed RoPE and the inverse
+    permutation.  Useful FLOPs: 2.5 x the forward's (five products per
+    visible pair: S, dP, dQ, dK, dV, against the forward's two)."""
+    from block_sparse_local_raster_b200 import ug
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl", world)
+    stream = torch.cuda.current_stream(dev)
+    plan = ug.Plan(**wl.geom_dict())
+    x = workloads.make_inputs(wl, seed=rank)
+    x.pop("head_scale", None)
+    x.update(workloads.make_grad_outputs(wl, seed=rank + 1))
+    d = {k: v.to(dev) for k, v in x.items()}
+    L = wl.n_lr
+    lr = lambda n: d[n] if L else None
+    o_hr, o_lr, lse = ug.layer_forward(plan, d["q_hr"], d["k_hr"], d["v_hr"], lr("q_lr"),
+                                       lr("k_lr"), lr("v_lr"))
+    B, N, H, Dh = d["q_hr"].shape
+    e = lambda t: torch.empty_like(t) if t is not None else None
+    wf = {n: torch.empty_like(d["q_hr"]) for n in ("q", "k", "v", "o", "do", "dq", "dk", "dv")}
+    ql_r, kl_r = e(lr("q_lr")), e(lr("k_lr"))
+    dq_hr, dk_hr, dv_hr = e(d["q_hr"]), e(d["k_hr"]), e(d["v_hr"])
+    dq_lr, dk_lr, dv_lr = e(lr("q_lr")), e(lr("k_lr")), e(lr("v_lr"))
+    aws = torch.empty(plan.attn_bwd_workspace_bytes(), dtype=torch.uint8, device=dev)
+
+    def chk(st, what):
+        if st != ug.UG_OK:
+            raise ug.UgError(st, what)
+
+    def step(ev=None):
+        chk(plan.permute_rope_window_first(d["q_hr"], wf["q"]), "q")
+        chk(plan.permute_rope_window_first(d["k_hr"], wf["k"]), "k")
+        chk(plan.permute_window_first(d["v_hr"], wf["v"]), "v")
+        chk(plan.permute_window_first(o_hr, wf["o"]), "o")
+        chk(plan.permute_window_first(d["do_hr"], wf["do"]), "do")
+        if L:
+            chk(plan.rope_2d(d["q_lr"], ql_r, ug.UG_LR), "q_lr")
+            chk(plan.rope_2d(d["k_lr"], kl_r, ug.UG_LR), "k_lr")
+        if ev is not None:
+            ev[0].record(stream)
+        chk(plan.hier_local_attn_bwd(wf["q"], wf["k"], wf["v"], ql_r, kl_r, lr("v_lr"), wf["o"],
+                                     o_lr, wf["do"], lr("do_lr"), lse, wf["dq"], wf["dk"],
+                                     wf["dv"], dq_lr, dk_lr, dv_lr, aws), "attention backward")
+        if ev is not None:
+            ev[1].record(stream)
+        chk(plan.unpermute_rope_bwd(wf["dq"], dq_hr), "dq")
+        chk(plan.unpermute_rope_bwd(wf["dk"], dk_hr), "dk")
+        chk(plan.unpermute(wf["dv"], dv_hr), "dv")
+        if L:
+            chk(plan.rope_2d_bwd(dq_lr, dq_lr, ug.UG_LR), "dq_lr")
+            chk(plan.rope_2d_bwd(dk_lr, dk_lr, ug.UG_LR), "dk_lr")
+
+    launches = 5 + (2 if L else 0) + 3 + 3 + (2 if L else 0)
+    flops = int(2.5 * useful_flops(wl))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    chk(plan.check_error(), "warm-up")
+    clocks = ClockSampler(local) if rank == 0 else None
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    chk(plan.check_error(), "timed steps")
+    sec = reduce_max(t0.elapsed_time(t1) / 1e3 / args.steps, dev)
+    attn = reduce_max(sum(a.elapsed_time(b) for a, b in ev) / 1e3 / args.steps, dev)
+    # end to end: inputs (q, k, v, o, lse, do) from pinned host memory, the
+    # gradients back to pinned host memory, through ug_layer_bwd
+    ws = torch.empty(plan.layer_bwd_workspace_bytes(), dtype=torch.uint8, device=dev)
+    host_in = {k: v.pin_memory() for k, v in x.items()}
+    host_in["o_hr"], host_in["lse"] = o_hr.cpu().pin_memory(), lse.cpu().pin_memory()
+    if L:
+        host_in["o_lr"] = o_lr.cpu().pin_memory()
+    dev_in = {"o_hr": o_hr, "lse": lse, **({"o_lr": o_lr} if L else {}), **d}
+    grads = [t for t in (dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr) if t is not None]
+    host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in grads]
+    e2e_steps = max(3, min(args.e2e_steps, args.steps))
+    torch.cuda.synchronize(dev)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        for k, v in host_in.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        chk(plan.layer_bwd(d["q_hr"], d["k_hr"], d["v_hr"], lr("q_lr"), lr("k_lr"), lr("v_lr"),
+                           o_hr, o_lr, lse, d["do_hr"], lr("do_lr"), dq_hr, dk_hr, dv_hr, dq_lr,
+                           dk_lr, dv_lr, ws, stream), "ug_layer_bwd")
+        for h, t in zip(host_out, grads):
+            h.copy_(t, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_sec = reduce_max(a0.elapsed_time(a1) / 1e3 / e2e_steps, dev)
+    if rank == 0:
+        pk, src = peaks()
+        ach = flops / attn / 1e12
+        line = {
+            "metric": "useful attention-backward TFLOP/s & ms per layer backward", "op": "backward",
+            "value": aggregate(flops, world, sec) / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "useful_flop_per_backward": flops,
+                       "l2": "inputs larger than L2, no flush"},
+            "attn_bwd_ms": attn * 1e3, "attn_bwd_tflops": ach,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops_sustained"],
+                         "traffic": None, "peak_source": src + " (sustained)",
+                         "executed_products_per_pair": 7},
+            "e2e": {"value": aggregate(flops, world, e2e_sec) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": sum(v.numel() * v.element_size()
+                                              for v in host_in.values()),
+                    "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in grads)},
+            "gpu_launches": launches * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_warm_start(args, world, rank, local):
+    """The warm-start kernel on the latent of the --config image size.
+    Algorithmic bytes per launch: the low-res latent read once, the noise
+    read once and the state written once (fp32).  The timed launches rotate
+    over enough noise/output buffers to exceed L2."""
+    from block_sparse_local_raster_b200 import ug
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl", world)
+    stream = torch.cuda.current_stream(dev)
+    ws = workloads.WARM_START[args.config]
+    host = workloads.make_warm_start_inputs(ws, seed=rank)
+    lr = host["x_lr"].to(dev)
+    hr_bytes = host["noise"].numel() * 4
+    nbuf = max(2, -(-3 * L2_BYTES // (2 * hr_bytes)))
+    noise = [host["noise"].to(dev) for _ in range(nbuf)]
+    outs = [torch.empty_like(noise[0]) for _ in range(nbuf)]
+    algo = lr.numel() * 4 + 2 * hr_bytes
+
+    def launch(i):
+        st = ug.warm_start_raw(lr, noise[i % nbuf], outs[i % nbuf], ws.scale, ws.sharpen, ws.t,
+                               stream)
+        if st != ug.UG_OK:
+            raise ug.UgError(st, "ug_warm_start")
+
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for i in range(args.steps):
+        launch(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    sec = reduce_max(e0.elapsed_time(e1) / 1e3 / args.steps, dev)
+    # end to end: pinned host buffers in, result out, every step
+    pin_lr, pin_noise = host["x_lr"].pin_memory(), host["noise"].pin_memory()
+    pin_out = torch.empty_like(pin_noise).pin_memory()
+    e2e_steps = max(3, min(args.e2e_steps, args.steps))
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(e2e_steps):
+        lr.copy_(pin_lr, non_blocking=True)
+        noise[0].copy_(pin_noise, non_blocking=True)
+        launch(0)
+        pin_out.copy_(outs[0], non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_sec = reduce_max(t0.elapsed_time(t1) / 1e3 / e2e_steps, dev)
+    pk, src = peaks()
+    if rank == 0:
+        gbs = algo / sec / 1e9
+        line = {
+            "metric": "warm-start initialisation HBM throughput", "op": "warm_start",
+            "value": aggregate(algo, world, sec) / 1e9, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": f"warm-start {ws.name}: [{ws.batch},{ws.channels},"
+                                   f"{ws.lr_h},{ws.lr_w}] x{ws.scale}, sharpen {ws.sharpen}, "
+                                   f"t {ws.t}", "l2": f"rotating {nbuf} buffer pairs > L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None, "peak_source": src,
+                         "algorithmic_bytes_per_launch": algo},
+            "e2e": {"value": aggregate(algo, world, e2e_sec) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": lr.numel() * 4 + hr_bytes,
+                    "d2h_bytes_per_step": hr_bytes},
+            "gpu_launches": args.steps, "clocks": clk,
+        }
+        if not args.no_cpu_baseline:
+            from oracle import warm_start as W
+            one = (slice(0, 1), slice(0, 1))
+            xs, ns = host["x_lr"][one].double().numpy(), host["noise"][one].double().numpy()
+            c0 = time.perf_counter()
+            W.warm_start(xs, ns, ws.scale, ws.sharpen, ws.t)
+            cdt = time.perf_counter() - c0
+            b1 = (xs.size + 2 * ns.size) * 4
+            line["cpu_baseline"] = {"value": b1 / cdt / 1e9, "unit": "GB/s", "cores": cpu_threads(),
+                                    "kind": "oracle",
+                                    "sample": f"one plane of the latent, fp64 numpy, {cdt:.2f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     world, rank, local = dist_env()
     if args.gpus != world and world > 1:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    if args.op == "warm_start":
+        if args.impl == "reference":
+            raise SystemExit("--op warm_start times the library only")
+        run_warm_start(args, world, rank, local)
+        return
+    if args.op == "backward":
+        if args.impl == "reference":
+            raise SystemExit("--op backward times the library only")
+        run_backward(args, workloads.get(args.config), world, rank, local)
+        return
     wl = workloads.get(args.config)
     if args.impl == "reference":
         run_reference(args, wl, world, rank)

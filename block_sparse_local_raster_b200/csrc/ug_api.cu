@@ -1,4 +1,5 @@
 // The C ABI: argument checks, plan lifetime, the layer sequence.
+#include <cmath>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -104,15 +105,19 @@ int ug_plan_create(const ug_geom* g, ug_plan** out) {
     build_neighbours(*g, p->nbr_off, p->nbr_idx);
     build_attention_lists(*g, p->nbr_off, p->nbr_idx, p->qtiles, p->kvlist, &p->n_hr_ctas,
                           &p->n_lr_ctas);
+    build_backward_lists(*g, p->nbr_off, p->nbr_idx, p->ktiles, p->qlist);
     std::vector<float> tables32;
     build_rope_tables(*g, p->rope, tables32);
     const std::vector<double> tables(tables32.begin(), tables32.end());
-    // One device block: [err (256 B)] [rope tables] [qtiles] [kvlist]
+    // One device block: [err (256 B)] [rope tables] [qtiles] [kvlist] [ktiles] [qlist]
     const size_t a_err = 0;
     const size_t a_rope = 256;
     const size_t a_qt = (a_rope + tables.size() * sizeof(double) + 255) / 256 * 256;
     const size_t a_kv = (a_qt + p->qtiles.size() * sizeof(QTile) + 255) / 256 * 256;
-    const size_t total = a_kv + std::max<size_t>(1, p->kvlist.size()) * sizeof(uint32_t);
+    const size_t a_kt = (a_kv + std::max<size_t>(1, p->kvlist.size()) * sizeof(uint32_t) + 255) /
+                        256 * 256;
+    const size_t a_ql = (a_kt + p->ktiles.size() * sizeof(KTile) + 255) / 256 * 256;
+    const size_t total = a_ql + std::max<size_t>(1, p->qlist.size()) * sizeof(uint32_t);
     if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return UG_ERR_CUDA; }
     if (cudaMalloc(&p->d_mem, total) != cudaSuccess) {
       cudaGetLastError();
@@ -124,10 +129,14 @@ int ug_plan_create(const ug_geom* g, ug_plan** out) {
     p->d_rope = reinterpret_cast<double*>(base + a_rope);
     p->d_qtiles = reinterpret_cast<QTile*>(base + a_qt);
     p->d_kvlist = reinterpret_cast<uint32_t*>(base + a_kv);
+    p->d_ktiles = reinterpret_cast<KTile*>(base + a_kt);
+    p->d_qlist = reinterpret_cast<uint32_t*>(base + a_ql);
     std::vector<char> host(total, 0);
     std::memcpy(host.data() + a_rope, tables.data(), tables.size() * sizeof(double));
     std::memcpy(host.data() + a_qt, p->qtiles.data(), p->qtiles.size() * sizeof(QTile));
     std::memcpy(host.data() + a_kv, p->kvlist.data(), p->kvlist.size() * sizeof(uint32_t));
+    std::memcpy(host.data() + a_kt, p->ktiles.data(), p->ktiles.size() * sizeof(KTile));
+    std::memcpy(host.data() + a_ql, p->qlist.data(), p->qlist.size() * sizeof(uint32_t));
     if (cudaMemcpy(p->d_mem, host.data(), total, cudaMemcpyHostToDevice) != cudaSuccess) {
       cudaFree(p->d_mem);
       delete p;
@@ -268,10 +277,162 @@ int ug_layer_fwd(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   return ug_unpermute(p, o_wf, o_hr, s);
 }
 
+// ---- backward ----------------------------------------------------------------
+
+int ug_rope_2d_bwd(const ug_plan* p, const void* dy, void* dx, int token_set, void* s) {
+  if (!p || !dy || !dx) return UG_ERR_INVALID_ARG;
+  if (token_set != UG_HR_WINDOW_FIRST && token_set != UG_HR_RASTER && token_set != UG_LR)
+    return UG_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(dx)) return UG_ERR_ALIGNMENT;
+  const int64_t n = token_set == UG_LR ? lr_bytes(p) : hr_bytes(p);
+  if (n == 0) return UG_OK;
+  if (dy != dx && overlap(dy, n, dx, n)) return UG_ERR_ALIAS;
+  return launch_rope(p, dy, dx, token_set, as_stream(s), true);
+}
+
+int ug_unpermute_rope_bwd(const ug_plan* p, const void* src_wf, void* dst_raster, void* s) {
+  if (!p || !src_wf || !dst_raster) return UG_ERR_INVALID_ARG;
+  if (!aligned16(src_wf) || !aligned16(dst_raster)) return UG_ERR_ALIGNMENT;
+  const int64_t n = hr_bytes(p);
+  if (overlap(src_wf, n, dst_raster, n)) return UG_ERR_ALIAS;
+  return launch_permute_rope(p, src_wf, dst_raster, as_stream(s), true);
+}
+
+int64_t ug_attn_bwd_workspace_bytes(const ug_plan* p) {
+  if (!p) return -1;
+  return ((int64_t)p->g.batch * p->g.heads * (p->N + p->L) * 4 + 255) / 256 * 256;
+}
+
+int ug_hier_local_attn_bwd(const ug_plan* p, const void* q_hr, const void* k_hr,
+                           const void* v_hr, const void* q_lr, const void* k_lr,
+                           const void* v_lr, const void* o_hr, const void* o_lr,
+                           const void* do_hr, const void* do_lr, const float* lse, void* dq_hr,
+                           void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr, void* dv_lr,
+                           void* workspace, int64_t workspace_bytes, void* s) {
+  if (!p || !lse || !workspace) return UG_ERR_INVALID_ARG;
+  if (workspace_bytes < ug_attn_bwd_workspace_bytes(p)) return UG_ERR_INVALID_ARG;
+  const bool lr = p->L > 0;
+  const void* ins[10] = {q_hr, k_hr, v_hr, o_hr, do_hr, q_lr, k_lr, v_lr, o_lr, do_lr};
+  void* outs[6] = {dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr};
+  for (int i = 0; i < 10; ++i)
+    if (!ins[i] && (i < 5 || lr)) return UG_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (!outs[i] && (i < 3 || lr)) return UG_ERR_INVALID_ARG;
+  if (p->g.head_dim != 64 && p->g.head_dim != 128) return UG_ERR_UNSUPPORTED;
+  for (const void* a : ins)
+    if (a && !aligned16(a)) return UG_ERR_ALIGNMENT;
+  for (const void* a : outs)
+    if (a && !aligned16(a)) return UG_ERR_ALIGNMENT;
+  if (!aligned16(lse) || !aligned16(workspace)) return UG_ERR_ALIGNMENT;
+  const int64_t nh = hr_bytes(p), nl = lr ? lr_bytes(p) : 0;
+  const int64_t nlse = (int64_t)p->g.batch * p->g.heads * (p->N + p->L) * 4;
+  const int64_t nws = ug_attn_bwd_workspace_bytes(p);
+  // every output and the workspace are disjoint from each other and from every input
+  const void* w[7] = {outs[0], outs[1], outs[2], outs[3], outs[4], outs[5], workspace};
+  const int64_t wn[7] = {nh, nh, nh, nl, nl, nl, nws};
+  for (int i = 0; i < 7; ++i) {
+    for (int j = 0; j < 10; ++j)
+      if (overlap(w[i], wn[i], ins[j], j < 5 ? nh : nl)) return UG_ERR_ALIAS;
+    if (overlap(w[i], wn[i], lse, nlse)) return UG_ERR_ALIAS;
+    for (int j = i + 1; j < 7; ++j)
+      if (overlap(w[i], wn[i], w[j], wn[j])) return UG_ERR_ALIAS;
+  }
+  return launch_attention_bwd(p, q_hr, k_hr, v_hr, lr ? q_lr : nullptr, lr ? k_lr : nullptr,
+                              lr ? v_lr : nullptr, o_hr, lr ? o_lr : nullptr, do_hr,
+                              lr ? do_lr : nullptr, lse, dq_hr, dk_hr, dv_hr,
+                              lr ? dq_lr : nullptr, lr ? dk_lr : nullptr, lr ? dv_lr : nullptr,
+                              static_cast<float*>(workspace), as_stream(s));
+}
+
+int64_t ug_layer_bwd_workspace_bytes(const ug_plan* p) {
+  if (!p) return -1;
+  auto up = [](int64_t n) { return (n + 255) / 256 * 256; };
+  return 8 * up(hr_bytes(p)) + 2 * up(lr_bytes(p)) + ug_attn_bwd_workspace_bytes(p);
+}
+
+int ug_layer_bwd(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+                 const void* q_lr, const void* k_lr, const void* v_lr, const void* o_hr,
+                 const void* o_lr, const float* lse, const void* do_hr, const void* do_lr,
+                 void* dq_hr, void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr, void* dv_lr,
+                 void* workspace, int64_t workspace_bytes, void* s) {
+  if (!p || !workspace) return UG_ERR_INVALID_ARG;
+  const int64_t ws = ug_layer_bwd_workspace_bytes(p);
+  if (workspace_bytes < ws) return UG_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return UG_ERR_ALIGNMENT;
+  const bool lr = p->L > 0;
+  const void* ins[10] = {q_hr, k_hr, v_hr, o_hr, do_hr, q_lr, k_lr, v_lr, o_lr, do_lr};
+  void* outs[6] = {dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr};
+  if (!lse) return UG_ERR_INVALID_ARG;
+  for (int i = 0; i < 10; ++i)
+    if (!ins[i] && (i < 5 || lr)) return UG_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (!outs[i] && (i < 3 || lr)) return UG_ERR_INVALID_ARG;
+  if (p->g.head_dim != 64 && p->g.head_dim != 128) return UG_ERR_UNSUPPORTED;
+  const int64_t nh = hr_bytes(p), nl = lr ? lr_bytes(p) : 0;
+  for (int i = 0; i < 10; ++i)
+    if (overlap(workspace, ws, ins[i], i < 5 ? nh : nl)) return UG_ERR_ALIAS;
+  for (int i = 0; i < 6; ++i)
+    if (overlap(workspace, ws, outs[i], i < 3 ? nh : nl)) return UG_ERR_ALIAS;
+  auto up = [](int64_t n) { return (n + 255) / 256 * 256; };
+  char* w = static_cast<char*>(workspace);
+  void* q_wf = w;
+  void* k_wf = w + up(nh);
+  void* v_wf = w + 2 * up(nh);
+  void* o_wf = w + 3 * up(nh);
+  void* do_wf = w + 4 * up(nh);
+  void* dq_wf = w + 5 * up(nh);
+  void* dk_wf = w + 6 * up(nh);
+  void* dv_wf = w + 7 * up(nh);
+  void* q_lr_r = w + 8 * up(nh);
+  void* k_lr_r = w + 8 * up(nh) + up(nl);
+  void* delta = w + 8 * up(nh) + 2 * up(nl);
+  int st;
+  if ((st = ug_permute_rope_window_first(p, q_hr, q_wf, s)) != UG_OK) return st;
+  if ((st = ug_permute_rope_window_first(p, k_hr, k_wf, s)) != UG_OK) return st;
+  if ((st = ug_permute_window_first(p, v_hr, v_wf, s)) != UG_OK) return st;
+  if ((st = ug_permute_window_first(p, o_hr, o_wf, s)) != UG_OK) return st;
+  if ((st = ug_permute_window_first(p, do_hr, do_wf, s)) != UG_OK) return st;
+  if (lr) {
+    if ((st = ug_rope_2d(p, q_lr, q_lr_r, UG_LR, s)) != UG_OK) return st;
+    if ((st = ug_rope_2d(p, k_lr, k_lr_r, UG_LR, s)) != UG_OK) return st;
+  }
+  // global dq, dk land in the outputs in the rotated frame, then rotate back in place
+  if ((st = ug_hier_local_attn_bwd(p, q_wf, k_wf, v_wf, q_lr_r, k_lr_r, v_lr, o_wf, o_lr, do_wf,
+                                   do_lr, lse, dq_wf, dk_wf, dv_wf, dq_lr, dk_lr, dv_lr, delta,
+                                   ug_attn_bwd_workspace_bytes(p), s)) != UG_OK)
+    return st;
+  if ((st = ug_unpermute_rope_bwd(p, dq_wf, dq_hr, s)) != UG_OK) return st;
+  if ((st = ug_unpermute_rope_bwd(p, dk_wf, dk_hr, s)) != UG_OK) return st;
+  if ((st = ug_unpermute(p, dv_wf, dv_hr, s)) != UG_OK) return st;
+  if (lr) {
+    if ((st = ug_rope_2d_bwd(p, dq_lr, dq_lr, UG_LR, s)) != UG_OK) return st;
+    if ((st = ug_rope_2d_bwd(p, dk_lr, dk_lr, UG_LR, s)) != UG_OK) return st;
+  }
+  return UG_OK;
+}
+
 int ug_plan_set_wait_timeout(ug_plan* p, int64_t ns) {
   if (!p || ns <= 0) return UG_ERR_INVALID_ARG;
   p->wait_timeout_ns = ns;
   return UG_OK;
+}
+
+int ug_warm_start(const ug_warm_start_params* q, const float* x_lr, const float* noise,
+                  float* out, void* s) {
+  if (!q || !x_lr || !noise || !out) return UG_ERR_INVALID_ARG;
+  if (q->batch < 1 || q->channels < 1 || q->lr_h < 1 || q->lr_w < 1 || q->scale < 1)
+    return UG_ERR_INVALID_ARG;
+  if ((int64_t)q->batch * q->channels > 65535) return UG_ERR_INVALID_ARG;
+  if ((int64_t)q->lr_h * q->scale > (1 << 24) || (int64_t)q->lr_w * q->scale > (1 << 24))
+    return UG_ERR_INVALID_ARG;
+  if (!std::isfinite(q->sharpen) || !(q->t >= 0.0f && q->t <= 1.0f)) return UG_ERR_INVALID_ARG;
+  if (!aligned16(x_lr) || !aligned16(noise) || !aligned16(out)) return UG_ERR_ALIGNMENT;
+  const int64_t planes = (int64_t)q->batch * q->channels;
+  const int64_t lo = planes * q->lr_h * q->lr_w * 4;
+  const int64_t hi = planes * ((int64_t)q->lr_h * q->scale) * ((int64_t)q->lr_w * q->scale) * 4;
+  if (overlap(out, hi, x_lr, lo)) return UG_ERR_ALIAS;
+  if (out != noise && overlap(out, hi, noise, hi)) return UG_ERR_ALIAS;
+  return launch_warm_start(q, x_lr, noise, out, as_stream(s));
 }
 
 int ug_check_error(const ug_plan* p, void* s) {

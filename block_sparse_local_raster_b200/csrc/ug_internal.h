@@ -27,6 +27,16 @@ struct QTile {
   int32_t list_len;  // number of key blocks (>= 1)
 };
 
+// One key CTA of the attention backward (dK, dV): its 128 keys, and its slice
+// of the query-tile list (the 128-row query tiles holding a query that sees
+// one of the keys).
+struct KTile {
+  int32_t lowres;    // 0: high-res keys (window-first), 1: global keys
+  int32_t k0;        // first key of the block inside its tensor
+  int32_t list_off;  // first entry in the query-tile list
+  int32_t list_len;  // number of query tiles (>= 1)
+};
+
 // Key-block list entry: block index (keys [128*idx, 128*idx + 128) of its
 // tensor), whether it lies in the low-res tensor, and whether some
 // (query, key) pair inside it is invisible or out of range so that the
@@ -65,6 +75,8 @@ struct ug_plan {
   std::vector<int32_t> perm, nbr_off, nbr_idx;
   std::vector<ug::QTile> qtiles;
   std::vector<uint32_t> kvlist;
+  std::vector<ug::KTile> ktiles;  // backward: key CTAs
+  std::vector<uint32_t> qlist;    // backward: query tiles per key CTA (entry format as kvlist)
   int32_t n_hr_ctas, n_lr_ctas;
   ug::RopeTables rope;
 
@@ -72,6 +84,8 @@ struct ug_plan {
   double* d_rope;          // RoPE tables
   ug::QTile* d_qtiles;     // attention query CTAs
   uint32_t* d_kvlist;      // attention key-block lists
+  ug::KTile* d_ktiles;     // backward key CTAs
+  uint32_t* d_qlist;       // backward query-tile lists
   int* d_err;              // first device-side error status (0 = none)
   int64_t wait_timeout_ns;
 };
@@ -85,12 +99,24 @@ void build_neighbours(const ug_geom& g, std::vector<int32_t>& off, std::vector<i
 void build_attention_lists(const ug_geom& g, const std::vector<int32_t>& nbr_off,
                            const std::vector<int32_t>& nbr_idx, std::vector<QTile>& qtiles,
                            std::vector<uint32_t>& kvlist, int32_t* n_hr_ctas, int32_t* n_lr_ctas);
+void build_backward_lists(const ug_geom& g, const std::vector<int32_t>& nbr_off,
+                          const std::vector<int32_t>& nbr_idx, std::vector<KTile>& ktiles,
+                          std::vector<uint32_t>& qlist);
 void build_rope_tables(const ug_geom& g, RopeTables& off, std::vector<float>& data);
 
 // Kernel launchers (one .cu each).  Arguments are already checked.
 int launch_permute(const ug_plan* p, const void* src, void* dst, bool inverse, cudaStream_t s);
-int launch_rope(const ug_plan* p, const void* x, void* y, int token_set, cudaStream_t s);
-int launch_permute_rope(const ug_plan* p, const void* src, void* dst, cudaStream_t s);
+int launch_rope(const ug_plan* p, const void* x, void* y, int token_set, cudaStream_t s,
+                bool transpose = false);
+int launch_permute_rope(const ug_plan* p, const void* src, void* dst, cudaStream_t s,
+                        bool inverse = false);
+int launch_attention_bwd(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+                         const void* q_lr, const void* k_lr, const void* v_lr, const void* o_hr,
+                         const void* o_lr, const void* do_hr, const void* do_lr, const float* lse,
+                         void* dq_hr, void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr,
+                         void* dv_lr, float* delta, cudaStream_t s);
+int launch_warm_start(const ug_warm_start_params* p, const float* x_lr, const float* noise,
+                      float* out, cudaStream_t s);
 int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                      const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
                      void* o_lr, float* lse, cudaStream_t s);

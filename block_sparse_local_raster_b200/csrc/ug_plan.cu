@@ -120,6 +120,61 @@ void build_attention_lists(const ug_geom& g, const std::vector<int32_t>& nbr_off
   *n_lr_ctas = nlr;
 }
 
+// Per 128-key block, the 128-row query tiles that see one of its keys.
+// Global key blocks come first (every query tile sees them: the longest
+// lists start earliest), then the high-res blocks, whose queries are those of
+// the windows neighbouring the block's windows (the neighbour relation is
+// symmetric).  An entry is flagged when some in-range (query, key) pair of
+// the tile and block is invisible; ranges past the end of a tensor need no
+// flag (the kernel zeroes those queries' probabilities and drops those keys).
+void build_backward_lists(const ug_geom& g, const std::vector<int32_t>& nbr_off,
+                          const std::vector<int32_t>& nbr_idx, std::vector<KTile>& ktiles,
+                          std::vector<uint32_t>& qlist) {
+  const int64_t N = (int64_t)g.grid_h * g.grid_w, L = global_tokens(g);
+  const int64_t T = (int64_t)g.win_h * g.win_w;
+  const int nwx = g.grid_w / g.win_w;
+  const int64_t BK = kKeysPerBlock, BQ = kRowsPerTile;
+  const int64_t n_hr_q = (N + BQ - 1) / BQ, n_lr_q = (L + BQ - 1) / BQ;
+  ktiles.clear();
+  qlist.clear();
+  auto near = [&](int64_t a, int64_t b) {  // window ids
+    return std::llabs(a / nwx - b / nwx) <= g.radius && std::llabs(a % nwx - b % nwx) <= g.radius;
+  };
+  for (int64_t kb = 0; kb * BK < L; ++kb) {
+    KTile t;
+    t.lowres = 1;
+    t.k0 = (int32_t)(kb * BK);
+    t.list_off = (int32_t)qlist.size();
+    for (int64_t qt = 0; qt < n_hr_q; ++qt) qlist.push_back((uint32_t)qt);
+    for (int64_t qt = 0; qt < n_lr_q; ++qt) qlist.push_back((uint32_t)qt | kBlockLowres);
+    t.list_len = (int32_t)qlist.size() - t.list_off;
+    ktiles.push_back(t);
+  }
+  for (int64_t kb = 0; kb * BK < N; ++kb) {
+    const int64_t k0 = kb * BK, k1 = std::min(N, k0 + BK);
+    const int64_t kw0 = k0 / T, kw1 = (k1 - 1) / T;  // key windows
+    std::set<int64_t> tiles;
+    for (int64_t kw = kw0; kw <= kw1; ++kw)
+      for (int32_t e = nbr_off[(size_t)kw]; e < nbr_off[(size_t)kw + 1]; ++e) {
+        const int64_t w = nbr_idx[(size_t)e];
+        for (int64_t qt = w * T / BQ; qt <= (w * T + T - 1) / BQ; ++qt) tiles.insert(qt);
+      }
+    KTile t;
+    t.lowres = 0;
+    t.k0 = (int32_t)k0;
+    t.list_off = (int32_t)qlist.size();
+    for (int64_t qt : tiles) {
+      const int64_t q0 = qt * BQ, q1 = std::min(N, q0 + BQ);
+      bool full = true;
+      for (int64_t qw = q0 / T; full && qw <= (q1 - 1) / T; ++qw)
+        for (int64_t kw = kw0; full && kw <= kw1; ++kw) full = near(qw, kw);
+      qlist.push_back((uint32_t)qt | (full ? 0u : kBlockMasked));
+    }
+    t.list_len = (int32_t)qlist.size() - t.list_off;
+    ktiles.push_back(t);
+  }
+}
+
 // f_k = theta^(-2k/a) (one pow in fp64); angle = position * f_k (one fp64
 // product); cos and sin from the C library in fp64, rounded to fp32.
 static void axis_table(const std::vector<double>& pos, int a, double theta, float* c, float* s) {

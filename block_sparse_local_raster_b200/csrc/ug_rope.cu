@@ -13,6 +13,9 @@
 // Boldo & Melquiond, "Emulation of FMA and correctly rounded sums: proved
 // algorithms using rounding to odd", IEEE Trans. Computers 2008).
 //
+// The backward pass rotates gradients by the transposed rotation: the same
+// c, s with s negated (exact), so it is reproducible in the same way.
+//
 // HBM-bound: 2 bytes moved per byte of tensor.  The rotation keeps the
 // fp32 <-> fp64 conversions (the slowest part of the arithmetic) to 4 per
 // channel pair.
@@ -55,10 +58,11 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t xw, double c, double s)
 }
 
 // Rotates one 16-byte chunk (4 channel pairs) with the table rows of its
-// position.  k: chunk index inside the head (8 channels per chunk).
+// position.  k: chunk index inside the head (8 channels per chunk).  sgn is
+// +1 (rotation) or -1 (its transpose).
 __device__ __forceinline__ uint4 rotate_chunk(uint4 v, int k, int ay_chunks, const double* cr,
                                               const double* sr, const double* cc,
-                                              const double* sc) {
+                                              const double* sc, double sgn) {
   const bool ax_row = k < ay_chunks;
   const double* cp = ax_row ? cr + k * 4 : cc + (k - ay_chunks) * 4;
   const double* sp = ax_row ? sr + k * 4 : sc + (k - ay_chunks) * 4;
@@ -67,10 +71,10 @@ __device__ __forceinline__ uint4 rotate_chunk(uint4 v, int k, int ay_chunks, con
   const double2 s01 = __ldg(reinterpret_cast<const double2*>(sp));
   const double2 s23 = __ldg(reinterpret_cast<const double2*>(sp) + 1);
   uint4 o;
-  o.x = rotate_pair(v.x, c01.x, s01.x);
-  o.y = rotate_pair(v.y, c01.y, s01.y);
-  o.z = rotate_pair(v.z, c23.x, s23.x);
-  o.w = rotate_pair(v.w, c23.y, s23.y);
+  o.x = rotate_pair(v.x, c01.x, sgn * s01.x);
+  o.y = rotate_pair(v.y, c01.y, sgn * s01.y);
+  o.z = rotate_pair(v.z, c23.x, sgn * s23.x);
+  o.w = rotate_pair(v.w, c23.y, sgn * s23.y);
   return o;
 }
 
@@ -90,6 +94,7 @@ struct RopeArgs {
   int32_t set;         // ug_token_set
   int32_t grid_w, win_h, win_w, nwx, T, lr_w;
   int32_t text_len;    // UG_LR: leading text rows, copied unrotated
+  double sgn;          // +1 rotation, -1 its transpose (backward)
 };
 
 // One warp per token row: lanes walk the row's 16-byte chunks (coalesced);
@@ -129,7 +134,7 @@ __global__ void __launch_bounds__(kThreads) rope_kernel(const RopeArgs a) {
     const uint4* __restrict__ xs = a.x + row * a.row_chunks;
     uint4* __restrict__ ys = a.y + row * a.row_chunks;
     for (int32_t c = lane; c < a.row_chunks; c += 32)
-      ys[c] = rotate_chunk(xs[c], c % hc, a.ay_chunks, cr, sr, cc, sc);
+      ys[c] = rotate_chunk(xs[c], c % hc, a.ay_chunks, cr, sr, cc, sc, a.sgn);
   }
 }
 
@@ -150,6 +155,7 @@ struct PermuteRopeArgs {
   int64_t n_tok;
   int32_t row_chunks, head_chunks, ay_chunks, my, mx;
   int32_t grid_h, grid_w, win_h, win_w, nwx, T;
+  bool inverse;  // false: raster -> window-first, rotated; true: window-first -> raster, transposed
 };
 
 template <int HEAD_CHUNKS>
@@ -163,8 +169,9 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermuteRop
     const int32_t wy = y / a.win_h, ly = y - wy * a.win_h;
     const int64_t r0 = (int64_t)y * a.grid_w + (int64_t)wx * a.win_w;
     const int64_t p0 = ((int64_t)wy * a.nwx + wx) * a.T + (int64_t)ly * a.win_w;
-    const uint4* __restrict__ s = a.src + (b * a.n_tok + r0) * a.row_chunks;
-    uint4* __restrict__ d = a.dst + (b * a.n_tok + p0) * a.row_chunks;
+    const uint4* __restrict__ s = a.src + (b * a.n_tok + (a.inverse ? p0 : r0)) * a.row_chunks;
+    uint4* __restrict__ d = a.dst + (b * a.n_tok + (a.inverse ? r0 : p0)) * a.row_chunks;
+    const double sgn = a.inverse ? -1.0 : 1.0;
     const double* cr = a.cos_r + (int64_t)y * a.my;
     const double* sr = a.sin_r + (int64_t)y * a.my;
 #pragma unroll 4
@@ -174,7 +181,8 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermuteRop
       const double* sc = a.sin_c + (int64_t)x * a.mx;
       for (int32_t rc = threadIdx.x; rc < a.row_chunks; rc += kThreads)
         d[tl * a.row_chunks + rc] =
-            rotate_chunk(__ldcs(s + tl * a.row_chunks + rc), rc % hc, a.ay_chunks, cr, sr, cc, sc);
+            rotate_chunk(__ldcs(s + tl * a.row_chunks + rc), rc % hc, a.ay_chunks, cr, sr, cc, sc,
+                         sgn);
     }
   }
 }
@@ -187,8 +195,10 @@ int grid_for(const ug_plan* p, int64_t want) {
 
 }  // namespace
 
-int launch_rope(const ug_plan* p, const void* x, void* y, int set, cudaStream_t st) {
+int launch_rope(const ug_plan* p, const void* x, void* y, int set, cudaStream_t st,
+                bool transpose) {
   RopeArgs a;
+  a.sgn = transpose ? -1.0 : 1.0;
   a.x = static_cast<const uint4*>(x);
   a.y = static_cast<uint4*>(y);
   const bool lr = set == UG_LR;
@@ -223,8 +233,10 @@ int launch_rope(const ug_plan* p, const void* x, void* y, int set, cudaStream_t 
   return cudaGetLastError() == cudaSuccess ? UG_OK : UG_ERR_CUDA;
 }
 
-int launch_permute_rope(const ug_plan* p, const void* src, void* dst, cudaStream_t st) {
+int launch_permute_rope(const ug_plan* p, const void* src, void* dst, cudaStream_t st,
+                        bool inverse) {
   PermuteRopeArgs a;
+  a.inverse = inverse;
   a.src = static_cast<const uint4*>(src);
   a.dst = static_cast<uint4*>(dst);
   const double* t = p->d_rope;

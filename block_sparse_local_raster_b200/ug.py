@@ -37,7 +37,9 @@ EXPORTS = (
     "ug_permute_window_first", "ug_permute_rope_window_first", "ug_unpermute", "ug_rope_2d",
     "ug_hier_local_attn_fwd",
     "ug_layer_workspace_bytes", "ug_layer_fwd", "ug_layer_fwd_static_scratch",
-    "ug_plan_set_wait_timeout", "ug_check_error",
+    "ug_plan_set_wait_timeout", "ug_check_error", "ug_warm_start",
+    "ug_rope_2d_bwd", "ug_unpermute_rope_bwd", "ug_attn_bwd_workspace_bytes",
+    "ug_hier_local_attn_bwd", "ug_layer_bwd_workspace_bytes", "ug_layer_bwd",
 )
 
 # Capacity of the static scratch of ug_layer_fwd_static_scratch (ug.h).
@@ -59,6 +61,14 @@ class ug_geom(ctypes.Structure):
         ("rope_dim_y", ctypes.c_int32), ("rope_dim_x", ctypes.c_int32),
         ("rope_theta", ctypes.c_double), ("softmax_scale", ctypes.c_float),
         ("text_len", ctypes.c_int32),
+    ]
+
+
+class ug_warm_start_params(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("channels", ctypes.c_int32), ("lr_h", ctypes.c_int32),
+        ("lr_w", ctypes.c_int32), ("scale", ctypes.c_int32), ("sharpen", ctypes.c_float),
+        ("t", ctypes.c_float),
     ]
 
 
@@ -97,6 +107,13 @@ def lib() -> ctypes.CDLL:
         "ug_layer_fwd_static_scratch": (I32, [P, P, P, P, P, P, P, P, P, P, P]),
         "ug_plan_set_wait_timeout": (I32, [P, I64]),
         "ug_check_error": (I32, [P, P]),
+        "ug_warm_start": (I32, [ctypes.POINTER(ug_warm_start_params), P, P, P, P]),
+        "ug_rope_2d_bwd": (I32, [P, P, P, I32, P]),
+        "ug_unpermute_rope_bwd": (I32, [P, P, P, P]),
+        "ug_attn_bwd_workspace_bytes": (I64, [P]),
+        "ug_hier_local_attn_bwd": (I32, [P] + [P] * 17 + [P, I64, P]),
+        "ug_layer_bwd_workspace_bytes": (I64, [P]),
+        "ug_layer_bwd": (I32, [P] + [P] * 17 + [P, I64, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -237,6 +254,38 @@ class Plan:
     def check_error(self, stream=None) -> int:
         return lib().ug_check_error(self.handle, _stream(stream))
 
+    # -- backward ----------------------------------------------------------------
+    def rope_2d_bwd(self, dy, dx, token_set: int, stream=None) -> int:
+        return lib().ug_rope_2d_bwd(self.handle, _ptr(dy), _ptr(dx), int(token_set),
+                                    _stream(stream))
+
+    def unpermute_rope_bwd(self, src_wf, dst_raster, stream=None) -> int:
+        return lib().ug_unpermute_rope_bwd(self.handle, _ptr(src_wf), _ptr(dst_raster),
+                                           _stream(stream))
+
+    def attn_bwd_workspace_bytes(self) -> int:
+        return int(lib().ug_attn_bwd_workspace_bytes(self.handle))
+
+    def layer_bwd_workspace_bytes(self) -> int:
+        return int(lib().ug_layer_bwd_workspace_bytes(self.handle))
+
+    def hier_local_attn_bwd(self, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr, do_lr,
+                            lse, dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr, workspace,
+                            stream=None) -> int:
+        args = (q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr, do_lr, lse, dq_hr, dk_hr,
+                dv_hr, dq_lr, dk_lr, dv_lr, workspace)
+        return lib().ug_hier_local_attn_bwd(
+            self.handle, *[_ptr(a) for a in args],
+            ctypes.c_int64(workspace.numel() * workspace.element_size()), _stream(stream))
+
+    def layer_bwd(self, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, do_hr, do_lr,
+                  dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr, workspace, stream=None) -> int:
+        args = (q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, do_hr, do_lr, dq_hr, dk_hr,
+                dv_hr, dq_lr, dk_lr, dv_lr, workspace)
+        return lib().ug_layer_bwd(
+            self.handle, *[_ptr(a) for a in args],
+            ctypes.c_int64(workspace.numel() * workspace.element_size()), _stream(stream))
+
 
 # ---- convenience wrappers (allocate outputs with torch, raise on errors) -----
 
@@ -276,6 +325,63 @@ def hier_local_attn_fwd(plan: Plan, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, want_lse
     _check(plan.hier_local_attn_fwd(q_hr, k_hr, v_hr, *lr, o_hr, o_lr, lse),
            "ug_hier_local_attn_fwd")
     return o_hr, o_lr, lse
+
+
+def _like(x):
+    return torch.empty_like(x) if x is not None and x.numel() else None
+
+
+def hier_local_attn_bwd(plan: Plan, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr,
+                        do_lr, lse):
+    """Gradients of hier_local_attn_fwd; returns (dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr)."""
+    outs = [_like(t) for t in (q_hr, k_hr, v_hr, q_lr, k_lr, v_lr)]
+    ws = torch.empty(plan.attn_bwd_workspace_bytes(), dtype=torch.uint8, device=q_hr.device)
+    _check(plan.hier_local_attn_bwd(q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr, do_lr,
+                                    lse, *outs, ws), "ug_hier_local_attn_bwd")
+    return tuple(outs)
+
+
+def layer_backward(plan: Plan, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, do_hr, do_lr,
+                   workspace=None):
+    """Gradients of layer_forward w.r.t. its raster inputs; returns
+    (dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr)."""
+    if workspace is None:
+        workspace = torch.empty(plan.layer_bwd_workspace_bytes(), dtype=torch.uint8,
+                                device=q_hr.device)
+    outs = [_like(t) for t in (q_hr, k_hr, v_hr, q_lr, k_lr, v_lr)]
+    _check(plan.layer_bwd(q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, do_hr, do_lr,
+                          *outs, workspace), "ug_layer_bwd")
+    return tuple(outs)
+
+
+def rope_2d_bwd(plan: Plan, dy: torch.Tensor, token_set: int) -> torch.Tensor:
+    out = torch.empty_like(dy)
+    _check(plan.rope_2d_bwd(dy, out, token_set), "ug_rope_2d_bwd")
+    return out
+
+
+def unpermute_rope_bwd(plan: Plan, x: torch.Tensor) -> torch.Tensor:
+    out = torch.empty_like(x)
+    _check(plan.unpermute_rope_bwd(x, out), "ug_unpermute_rope_bwd")
+    return out
+
+
+def warm_start_raw(x_lr: torch.Tensor, noise: torch.Tensor, out: torch.Tensor, scale: int,
+                   sharpen: float, t: float, stream=None) -> int:
+    """ug_warm_start on fp32 [B, C, h, w] / [B, C, h*s, w*s] device tensors;
+    returns the status."""
+    B, C, h, w = x_lr.shape
+    prm = ug_warm_start_params(B, C, h, w, int(scale), float(sharpen), float(t))
+    return lib().ug_warm_start(ctypes.byref(prm), _ptr(x_lr), _ptr(noise), _ptr(out),
+                               _stream(stream))
+
+
+def warm_start(x_lr: torch.Tensor, noise: torch.Tensor, scale: int, sharpen: float, t: float,
+               out: torch.Tensor = None) -> torch.Tensor:
+    """(1 - t) * sharpen(upsample(x_lr)) + t * noise, into a new tensor (or out)."""
+    out = torch.empty_like(noise) if out is None else out
+    _check(warm_start_raw(x_lr, noise, out, scale, sharpen, t), "ug_warm_start")
+    return out
 
 
 def layer_forward(plan: Plan, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, workspace=None, want_lse=True):

@@ -161,6 +161,20 @@ def make_inputs(wl: Workload, seed: int = 0,
     return out
 
 
+def make_grad_outputs(wl: Workload, seed: int = 1,
+                      device: Optional[str] = None) -> Dict[str, torch.Tensor]:
+    """Seeded output gradients for the backward pass: do_hr [B, N, h, d] and
+    do_lr [B, L, h, d], i.i.d. N(0, 1) drawn in that order, rounded to bf16."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    out = {}
+    for name, n in (("do_hr", wl.n_hr), ("do_lr", wl.n_lr)):
+        t = torch.randn((wl.batch, n, wl.heads, wl.head_dim), generator=g, dtype=torch.float32)
+        out[name] = t.to(torch.bfloat16).contiguous()
+    if device is not None:
+        out = {k: v.to(device) for k, v in out.items()}
+    return out
+
+
 def make_tensor(shape, seed: int, scale: float = 1.0) -> torch.Tensor:
     """One seeded N(0, scale^2) bf16 tensor (CPU), for single-kernel tests."""
     g = torch.Generator(device="cpu").manual_seed(seed)
@@ -168,3 +182,45 @@ def make_tensor(shape, seed: int, scale: float = 1.0) -> torch.Tensor:
     if scale != 1.0:
         t.mul_(scale)
     return t.to(torch.bfloat16).contiguous()
+
+
+# Warm-start initialisation: FLUX-class latents have 16 channels at 1/8 of
+# the image size (two latent pixels per token side), so the 4K image is a
+# 16 x 512 x 512 latent and its low-res guidance (the 64 x 64 token grid) a
+# 16 x 128 x 128 one: factor 4 = rho.  The sharpening amount and the timestep
+# are not given on the pages; 0.5 and 0.6 stand in.
+@dataclasses.dataclass(frozen=True)
+class WarmStart:
+    name: str
+    batch: int
+    channels: int
+    lr_h: int
+    lr_w: int
+    scale: int
+    sharpen: float = 0.5
+    t: float = 0.6
+
+    @property
+    def hr_shape(self):
+        return (self.batch, self.channels, self.lr_h * self.scale, self.lr_w * self.scale)
+
+    @property
+    def lr_shape(self):
+        return (self.batch, self.channels, self.lr_h, self.lr_w)
+
+
+WARM_START: Dict[str, WarmStart] = {
+    "4K": WarmStart("4K", 1, 16, 128, 128, 4),
+    "8K": WarmStart("8K", 1, 16, 256, 256, 4),
+    "odd": WarmStart("odd", 2, 3, 13, 7, 3, sharpen=1.25, t=0.3),
+    "s1": WarmStart("s1", 1, 2, 9, 20, 1),
+    "wide": WarmStart("wide", 1, 1, 3, 70, 4, sharpen=0.0, t=0.0),
+}
+
+
+def make_warm_start_inputs(ws: WarmStart, seed: int = 0) -> Dict[str, torch.Tensor]:
+    """x_lr then noise, i.i.d. N(0, 1) fp32 from one seeded CPU generator."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    x_lr = torch.randn(ws.lr_shape, generator=g, dtype=torch.float32)
+    noise = torch.randn(ws.hr_shape, generator=g, dtype=torch.float32)
+    return {"x_lr": x_lr, "noise": noise}

@@ -242,6 +242,97 @@ int ug_layer_fwd_static_scratch(const ug_plan* plan, const void* q_hr, const voi
                                 const void* v_lr, void* o_hr, void* o_lr, float* lse,
                                 void* stream);
 
+/* ---- backward pass ------------------------------------------------------------
+ * Gradients of the layer for training (the pages train LoRA adapters on the
+ * q/k/v projections of the low-res guidance: UltraGen-ar §2.ج, UltraGen-fr
+ * §2.C).  With P the forward's probabilities (recomputed from its lse),
+ * D = rowsum(dO * O), dP = dO V^T and dS = P * (dP - D):
+ *   dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO;
+ * RoPE's gradient is the transposed rotation; the permutation's is its
+ * inverse.  bf16 in and out, fp32 accumulation; P and dS are rounded to bf16
+ * as tensor-core operands. */
+
+/* Transposed rotation of ug_rope_2d (the same fp32 cos/sin, sine negated):
+ * dx = R^T dy per channel pair, bit-reproducible like ug_rope_2d.  dy == dx
+ * is allowed; text rows of UG_LR are copied. */
+int ug_rope_2d_bwd(const ug_plan* plan, const void* dy, void* dx, int token_set, void* stream);
+
+/* The inverse of ug_permute_rope_window_first for gradients:
+ * dst_raster[b, r] = R^T(src_wf[b, perm[r]]) at raster token r's position,
+ * in one pass.  UG_ERR_ALIAS if the ranges overlap. */
+int ug_unpermute_rope_bwd(const ug_plan* plan, const void* src_wf, void* dst_raster,
+                          void* stream);
+
+/* Device scratch of ug_hier_local_attn_bwd: D, fp32 [B, h, N + L]. */
+int64_t ug_attn_bwd_workspace_bytes(const ug_plan* plan);
+
+/* Gradients of ug_hier_local_attn_fwd.  Inputs as its inputs (rotated q, k;
+ * high-res window-first), plus its outputs o_hr/o_lr and lse (required), and
+ * the output gradients do_hr [B, N, h, d] (window-first) and do_lr
+ * [B, L, h, d].  Outputs dq/dk/dv in the layouts of q/k/v (the *_lr ones
+ * ignored, may be NULL, if L = 0).  workspace: device, 16-byte aligned, at
+ * least ug_attn_bwd_workspace_bytes.  Outputs and workspace may not overlap
+ * each other or any input (UG_ERR_ALIAS).  d in {64, 128}.  Device waits are
+ * bounded as in the forward (UG_ERR_TIMEOUT via ug_check_error); a device
+ * whose dynamic shared memory is not 1024-byte aligned makes the dK/dV
+ * kernel record UG_ERR_UNSUPPORTED. */
+int ug_hier_local_attn_bwd(const ug_plan* plan, const void* q_hr, const void* k_hr,
+                           const void* v_hr, const void* q_lr, const void* k_lr,
+                           const void* v_lr, const void* o_hr, const void* o_lr,
+                           const void* do_hr, const void* do_lr, const float* lse, void* dq_hr,
+                           void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr, void* dv_lr,
+                           void* workspace, int64_t workspace_bytes, void* stream);
+
+/* Device scratch of ug_layer_bwd. */
+int64_t ug_layer_bwd_workspace_bytes(const ug_plan* plan);
+
+/* Gradients of ug_layer_fwd with respect to its raster-order inputs: given
+ * the layer's inputs q/k/v, its outputs o_hr (raster) / o_lr and lse, and
+ * do_hr (raster) / do_lr, writes dq/dk/dv (same layouts as q/k/v; dq, dk
+ * are gradients w.r.t. the unrotated q, k).  Recomputes the window-first,
+ * rotated operands, runs ug_hier_local_attn_bwd, then the inverse
+ * permutation with the transposed RoPE.  workspace: at least
+ * ug_layer_bwd_workspace_bytes, 256-byte aligned, disjoint from every
+ * argument. */
+int ug_layer_bwd(const ug_plan* plan, const void* q_hr, const void* k_hr, const void* v_hr,
+                 const void* q_lr, const void* k_lr, const void* v_lr, const void* o_hr,
+                 const void* o_lr, const float* lse, const void* do_hr, const void* do_lr,
+                 void* dq_hr, void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr, void* dv_lr,
+                 void* workspace, int64_t workspace_bytes, void* stream);
+
+/* ---- warm-start initialisation -------------------------------------------- */
+
+/* Sizes and constants of ug_warm_start. */
+typedef struct ug_warm_start_params {
+  int32_t batch;     /* B >= 1                                               */
+  int32_t channels;  /* C >= 1 latent channels; B * C <= 65535               */
+  int32_t lr_h;      /* low-res latent h x w, >= 1                            */
+  int32_t lr_w;
+  int32_t scale;     /* integer factor s >= 1: the high-res latent is        */
+                     /* (h*s) x (w*s), each side at most 2^24                */
+  float sharpen;     /* unsharp-mask amount (finite; 0 = no sharpening)      */
+  float t;           /* timestep in [0, 1]: 0 = the sharpened upsample,      */
+                     /* 1 = pure noise                                        */
+} ug_warm_start_params;
+
+/* Warm-start of the high-res state (UltraGen-ar §2.د "Warm-Start
+ * Initialization": the low-res guidance is upsampled, sharpened and added to
+ * the high-res representation at an intermediate timestep; UltraGen-fr §2.D:
+ * Gaussian noise combined with the upscaled low-res image).  Per plane of
+ * x_lr [B, C, h, w] fp32:
+ *   u   = bilinear upsampling by s with half-pixel centres: high-res pixel
+ *         (y, x) samples ((y + 0.5)/s - 0.5, (x + 0.5)/s - 0.5), low-res
+ *         indices clamped to the image;
+ *   x0  = u + sharpen * (u - blur(u)), blur the 3x3 binomial filter
+ *         (1/4, 1/2, 1/4) per axis with edges replicated;
+ *   out = (1 - t) * x0 + t * noise           (rectified-flow interpolation).
+ * noise and out: [B, C, h*s, w*s] fp32, device, 16-byte aligned; the caller
+ * draws the noise.  out == noise is allowed (in place); any other overlap of
+ * out with an input is UG_ERR_ALIAS.  fp32 arithmetic: within a few fp32
+ * ulps of the exact value.  No plan is needed. */
+int ug_warm_start(const ug_warm_start_params* params, const float* x_lr, const float* noise,
+                  float* out, void* stream);
+
 /* ---- errors ---------------------------------------------------------------- */
 
 /* Bound, in ns, on each device-side wait of this plan's attention kernel

@@ -82,3 +82,83 @@ def err_stats(got: np.ndarray, ref: np.ndarray, v_scale=None):
     d = d / s
     dmax = np.maximum(d - 2.0 ** -8 * np.abs(ref) / s, 0.0)
     return float(dmax.max()), float(d.mean())
+
+
+# ----------------------------------------------------------------- backward
+
+U = 2.0 ** -9  # unit roundoff of bf16 (8-bit significand)
+
+
+def bwd_error_bounds(g: O.Geometry, hr_order: str, q, k, v, do, rows=None, keys=None,
+                     heads=None, chunk_rows: int = 512):
+    """Per-element bounds on |GPU - exact| for dQ (rows) and dK, dV (keys).
+
+    q, k, v, do: joint-sequence fp64 arrays [B, n, h, d] (the bf16 inputs
+    widened).  The kernels round P and dS to bf16 as tensor-core operands
+    (relative U each), compute D = rowsum(dO * O) from the bf16 forward output
+    (relative U per product, so |dD| <= 2U sum |dO O| with the fp32 sum), sum
+    in fp32 and round every output to bf16 (U |result|).  With these:
+      |e dV_j| <= 2U sum_i P_ij |dO_i| + U |dV_j|
+      |e dS_ij| <= 2U |dS_ij| + P_ij |dD_i|
+      |e dQ_i| <= scale sum_j |e dS_ij| |K_j| + U |dQ_i|, likewise dK with Q.
+    Each bound is doubled (fp32 accumulation and the approximate exp2 are far
+    below it) and floored at 1e-6.  Returns (bq, bk, bv) shaped like the
+    oracle's attention_backward outputs."""
+    B, n, H, d = q.shape
+    rows = np.arange(n) if rows is None else np.asarray(rows, np.int64)
+    keys = np.arange(n) if keys is None else np.asarray(keys, np.int64)
+    heads = range(H) if heads is None else heads
+    need = np.union1d(rows, O.rows_seeing(g, hr_order, keys)) if keys.size else rows
+    pos = {int(r): i for i, r in enumerate(rows)}
+    bq = np.zeros((B, rows.size, H, d))
+    bk = np.zeros((B, keys.size, H, d))
+    bv = np.zeros((B, keys.size, H, d))
+    gq = np.zeros_like(bq)
+    gk = np.zeros_like(bk)
+    gv = np.zeros_like(bv)
+    for b in range(B):
+        for h in heads:
+            Q, K, V, dO = q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h]
+            for i0 in range(0, need.size, chunk_rows):
+                r = need[i0:i0 + chunk_rows]
+                s = (Q[r] @ K.T) * g.scale
+                s[~O.visibility(g, hr_order, r)] = -np.inf
+                p = np.exp(s - s.max(axis=1, keepdims=True))
+                p /= p.sum(axis=1, keepdims=True)
+                o = p @ V
+                dP = dO[r] @ V.T
+                D = (p * dP).sum(axis=1, keepdims=True)
+                dS = p * (dP - D)
+                dD = 2 * U * (np.abs(dO[r]) * np.abs(o)).sum(axis=1, keepdims=True)
+                eS = 2 * U * np.abs(dS) + p * dD
+                eq = g.scale * (eS @ np.abs(K))
+                gq_c = g.scale * (dS @ K)
+                for j, ri in enumerate(r):
+                    t = pos.get(int(ri))
+                    if t is not None:
+                        bq[b, t, h] = eq[j]
+                        gq[b, t, h] = gq_c[j]
+                bk[b, :, h] += g.scale * (eS.T @ np.abs(Q[r]))[keys]
+                gk[b, :, h] += g.scale * (dS.T @ Q[r])[keys]
+                bv[b, :, h] += 2 * U * (p.T @ np.abs(dO[r]))[keys]
+                gv[b, :, h] += (p.T @ dO[r])[keys]
+    fin = lambda e, gg: 2 * (e + U * np.abs(gg)) + 1e-6
+    return fin(bq, gq), fin(bk, gk), fin(bv, gv)
+
+
+def joint_f64(x: dict, name: str, heads=None) -> np.ndarray:
+    """[B, N + L, h, d] fp64 from the bf16 tensors name_hr, name_lr (only the
+    listed heads, in that order, if given)."""
+    sel = (lambda t: t) if heads is None else (lambda t: t[:, :, list(heads)])
+    hr = f64(sel(x[name + "_hr"]))
+    lr = f64(sel(x[name + "_lr"])) if x.get(name + "_lr") is not None else hr[:, :0]
+    return np.concatenate([hr, lr], axis=1)
+
+
+def rotated_bound(b: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """Bound after the transposed RoPE and its bf16 rounding: a rotation moves
+    an error pair (e0, e1) to components of size at most |(e0, e1)| <=
+    sqrt(2) max(b0, b1); the rounding adds U |ref|."""
+    m = np.maximum(b[..., 0::2], b[..., 1::2])
+    out = np.repeat(m, 2, axis=-1) * np.sqrt(2.0)
+    return out + U * np.abs(ref)

@@ -1,0 +1,205 @@
+"""GPU parity of the backward pass (attention, RoPE, whole layer) against the
+fp64 oracle, called through the C ABI.
+
+RoPE's transposed rotation and the inverse permutation are bit-exact.  The
+attention gradients are held to per-element bounds derived from the kernels'
+arithmetic (bf16 rounding of P and dS as tensor-core operands, of the forward
+output used for D, and of every output; fp32 sums): see
+``parity.bwd_error_bounds``.  Small geometries check every element; the 4K
+layer checks sampled query rows and high-res keys for two heads, and for all
+heads the identities sum_j dV_j = sum_i dO_i and sum_j dK_j = 0.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_local_raster_b200 import ug, workloads
+from oracle import hier_local_attn as O
+
+from parity import (U, bits, bwd_error_bounds, f64, joint_f64, ogeom, plan, rotated_bound,
+                    sample_hr_tokens, sample_lr_tokens)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+SMALL = list(workloads.TEST_GEOMETRIES) + ["tiny"]
+
+
+def inputs(wl, seed):
+    x = workloads.make_inputs(wl, seed=seed)
+    x.pop("head_scale", None)
+    x.update(workloads.make_grad_outputs(wl, seed=seed + 1))
+    return x
+
+
+def forward_backward(p, wl, d):
+    has_lr = wl.n_lr > 0
+    g = lambda n: d[n] if has_lr else None
+    o_hr, o_lr, lse = ug.hier_local_attn_fwd(p, d["q_hr"], d["k_hr"], d["v_hr"], g("q_lr"),
+                                             g("k_lr"), g("v_lr"))
+    grads = ug.hier_local_attn_bwd(p, d["q_hr"], d["k_hr"], d["v_hr"], g("q_lr"), g("k_lr"),
+                                   g("v_lr"), o_hr, o_lr, d["do_hr"], g("do_lr"), lse)
+    torch.cuda.synchronize()
+    assert p.check_error() == ug.UG_OK
+    return grads
+
+
+def joint_grads(grads, wl, heads=None):
+    sel = (lambda t: t) if heads is None else (lambda t: t[:, :, list(heads)])
+    out = []
+    for i in range(3):
+        hr = f64(sel(grads[i]))
+        lr = f64(sel(grads[3 + i])) if grads[3 + i] is not None else hr[:, :0]
+        out.append(np.concatenate([hr, lr], axis=1))
+    return out
+
+
+def check(got, ref, bound, what):
+    excess = np.abs(got - ref) - bound
+    worst = np.unravel_index(np.argmax(excess), excess.shape)
+    assert excess.max() <= 0, (what, float(excess.max()), float(np.abs(got - ref)[worst]),
+                               float(bound[worst]), worst)
+    return float(np.abs(got - ref).max())
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_attention_backward_every_element(name):
+    wl = workloads.get(name)
+    g = ogeom(wl)
+    p = plan(wl)
+    x = inputs(wl, 800)
+    grads = forward_backward(p, wl, {k: v.to(DEV) for k, v in x.items()})
+    xb = {k: bits(v) for k, v in x.items()}
+    ref = O.attention_backward(xb["q_hr"], xb["k_hr"], xb["v_hr"], xb["q_lr"], xb["k_lr"],
+                               xb["v_lr"], xb["do_hr"], xb["do_lr"], g, O.HR_WINDOW_FIRST)
+    bnd = bwd_error_bounds(g, O.HR_WINDOW_FIRST, *(joint_f64(x, n) for n in ("q", "k", "v", "do")))
+    for what, got, r, b in zip(("dq", "dk", "dv"), joint_grads(grads, wl), ref, bnd):
+        check(got, r, b, f"{name} {what}")
+
+
+def test_attention_backward_sampled_4k():
+    wl = workloads.get("4K")
+    g = ogeom(wl)
+    p = plan(wl)
+    x = inputs(wl, 810)
+    grads = forward_backward(p, wl, {k: v.to(DEV) for k, v in x.items()})
+    heads = [0, 23]
+    rows = np.concatenate([sample_hr_tokens(g, O.HR_WINDOW_FIRST, 5, n_interior=2, per_window=2),
+                           g.N + sample_lr_tokens(g, 5, n=4)])
+    T, nx = g.T, g.n_win_x
+    keys = np.array([0, T - 1, (7 * nx + 9) * T + 100, g.N - 1])  # corner, interior, last window
+    xb = {k: bits(v[:, :, heads]) for k, v in x.items()}
+    g1 = O.Geometry.from_dict(dict(wl.geom_dict(), heads=len(heads)))
+    ref = O.attention_backward(xb["q_hr"], xb["k_hr"], xb["v_hr"], xb["q_lr"], xb["k_lr"],
+                               xb["v_lr"], xb["do_hr"], xb["do_lr"], g1, O.HR_WINDOW_FIRST,
+                               rows=rows, keys=keys)
+    bnd = bwd_error_bounds(g1, O.HR_WINDOW_FIRST,
+                           *(joint_f64(x, n, heads) for n in ("q", "k", "v", "do")),
+                           rows=rows, keys=keys)
+    gq, gk, gv = joint_grads(grads, wl, heads)
+    check(gq[:, rows], ref[0], bnd[0], "4K dq")
+    check(gk[:, keys], ref[1], bnd[1], "4K dk")
+    check(gv[:, keys], ref[2], bnd[2], "4K dv")
+    # identities of any softmax attention, all heads, every key
+    gq, gk, gv = joint_grads(grads, wl)
+    do = joint_f64(x, "do")
+    assert np.all(np.abs(gv.sum(1) - do.sum(1)) <= 2 * U * np.abs(gv).sum(1) + 1e-3)
+    assert np.all(np.abs(gk.sum(1)) <= 4 * U * np.abs(gk).sum(1) + 1e-3)
+
+
+SETS = [(ug.UG_HR_WINDOW_FIRST, O.HR_WINDOW_FIRST), (ug.UG_HR_RASTER, O.HR_RASTER),
+        (ug.UG_LR, O.LOWRES)]
+
+
+@pytest.mark.parametrize("name", SMALL + ["4K"])
+def test_rope_backward_bit_exact(name):
+    wl = workloads.get(name)
+    g = ogeom(wl)
+    p = plan(wl)
+    tab = O.rope_tables(g)
+    for k, (uset, oset) in enumerate(SETS):
+        n = wl.n_lr if uset == ug.UG_LR else wl.n_hr
+        if n == 0:
+            continue
+        x = workloads.make_tensor((wl.batch, n, wl.heads, wl.head_dim), 900 + k)
+        y = ug.rope_2d_bwd(p, x.to(DEV), uset)
+        heads = range(wl.heads) if name != "4K" else [0, 13]
+        xb, yb = bits(x), bits(y)
+        for h in heads:
+            want = O.rope_2d_backward(xb[:, :, h:h + 1], g, oset, tables=tab)
+            np.testing.assert_array_equal(yb[:, :, h:h + 1], want, err_msg=f"{name} {oset} {h}")
+    assert p.check_error() == ug.UG_OK
+
+
+@pytest.mark.parametrize("name", SMALL + ["4K"])
+def test_unpermute_rope_backward_bit_exact(name):
+    wl = workloads.get(name)
+    g = ogeom(wl)
+    p = plan(wl)
+    x = workloads.make_tensor((wl.batch, wl.n_hr, wl.heads, wl.head_dim), 950)
+    y = ug.unpermute_rope_bwd(p, x.to(DEV))
+    xb, yb = bits(x), bits(y)
+    heads = range(wl.heads) if name != "4K" else [0, 13]
+    for h in heads:
+        want = O.unpermute(O.rope_2d_backward(xb[:, :, h:h + 1], g, O.HR_WINDOW_FIRST), g)
+        np.testing.assert_array_equal(yb[:, :, h:h + 1], want, err_msg=f"{name} {h}")
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_layer_backward_every_element(name):
+    """ug_layer_bwd on raster inputs against the oracle's layer gradients."""
+    wl = workloads.get(name)
+    g = ogeom(wl)
+    p = plan(wl)
+    x = inputs(wl, 820)
+    d = {k: v.to(DEV) for k, v in x.items()}
+    has_lr = wl.n_lr > 0
+    lr = lambda n: d[n] if has_lr else None
+    o_hr, o_lr, lse = ug.layer_forward(p, d["q_hr"], d["k_hr"], d["v_hr"], lr("q_lr"),
+                                       lr("k_lr"), lr("v_lr"))
+    grads = ug.layer_backward(p, d["q_hr"], d["k_hr"], d["v_hr"], lr("q_lr"), lr("k_lr"),
+                              lr("v_lr"), o_hr, o_lr, lse, d["do_hr"], lr("do_lr"))
+    torch.cuda.synchronize()
+    assert p.check_error() == ug.UG_OK
+    for k in d:  # inputs untouched
+        assert torch.equal(d[k].cpu(), x[k]), k
+    xb = {k: bits(v) for k, v in x.items()}
+    ref = O.layer_backward(xb, xb, g)
+    # bounds in the rotated frame (raster order), then through R^T for dq, dk
+    rot = {"q": np.concatenate([O.bf16_to_f64(O.rope_2d(xb["q_hr"], g, O.HR_RASTER)),
+                                O.bf16_to_f64(O.rope_2d(xb["q_lr"], g, O.LOWRES))], axis=1),
+           "k": np.concatenate([O.bf16_to_f64(O.rope_2d(xb["k_hr"], g, O.HR_RASTER)),
+                                O.bf16_to_f64(O.rope_2d(xb["k_lr"], g, O.LOWRES))], axis=1)}
+    bq, bk, bv = bwd_error_bounds(g, O.HR_RASTER, rot["q"], rot["k"], joint_f64(x, "v"),
+                                  joint_f64(x, "do"))
+    got = joint_grads(grads, wl)
+    check(got[0], ref[0], rotated_bound(bq, ref[0]), f"{name} layer dq")
+    check(got[1], ref[1], rotated_bound(bk, ref[1]), f"{name} layer dk")
+    check(got[2], ref[2], bv, f"{name} layer dv")
+
+
+def test_backward_error_statuses():
+    wl = workloads.get("tiny")
+    p = plan(wl)
+    x = {k: v.to(DEV) for k, v in inputs(wl, 830).items()}
+    o_hr, o_lr, lse = ug.hier_local_attn_fwd(p, x["q_hr"], x["k_hr"], x["v_hr"], x["q_lr"],
+                                             x["k_lr"], x["v_lr"])
+    outs = [torch.empty_like(x[n]) for n in ("q_hr", "k_hr", "v_hr", "q_lr", "k_lr", "v_lr")]
+    ws = torch.empty(p.attn_bwd_workspace_bytes(), dtype=torch.uint8, device=DEV)
+    args = lambda **kw: [kw.get(n, v) for n, v in (
+        ("q_hr", x["q_hr"]), ("k_hr", x["k_hr"]), ("v_hr", x["v_hr"]), ("q_lr", x["q_lr"]),
+        ("k_lr", x["k_lr"]), ("v_lr", x["v_lr"]), ("o_hr", o_hr), ("o_lr", o_lr),
+        ("do_hr", x["do_hr"]), ("do_lr", x["do_lr"]), ("lse", lse), ("dq_hr", outs[0]),
+        ("dk_hr", outs[1]), ("dv_hr", outs[2]), ("dq_lr", outs[3]), ("dk_lr", outs[4]),
+        ("dv_lr", outs[5]), ("ws", ws))]
+    assert p.hier_local_attn_bwd(*args()) == ug.UG_OK
+    assert p.hier_local_attn_bwd(*args(lse=None)) == ug.UG_ERR_INVALID_ARG
+    assert p.hier_local_attn_bwd(*args(dq_hr=x["q_hr"])) == ug.UG_ERR_ALIAS
+    assert p.hier_local_attn_bwd(*args(dk_hr=outs[0])) == ug.UG_ERR_ALIAS
+    assert p.hier_local_attn_bwd(*args(ws=ws[:16])) == ug.UG_ERR_INVALID_ARG
+    flat = torch.empty(outs[0].numel() + 8, dtype=torch.bfloat16, device=DEV)
+    assert p.hier_local_attn_bwd(*args(dq_hr=flat[1:1 + outs[0].numel()].view_as(outs[0]))) \
+        == ug.UG_ERR_ALIGNMENT
+    assert p.rope_2d_bwd(x["q_hr"], x["q_hr"], 9) == ug.UG_ERR_INVALID_ARG
+    assert p.unpermute_rope_bwd(x["q_hr"], x["q_hr"]) == ug.UG_ERR_ALIAS
+    torch.cuda.synchronize()
+    assert p.check_error() == ug.UG_OK
