@@ -52,29 +52,52 @@ __device__ __forceinline__ void taps(int d, int s, int n, int& i0, int& i1, floa
 template <bool VEC>
 __global__ void __launch_bounds__(kThreads) warm_start_kernel(const WarmArgs a) {
   __shared__ float u[kUH][kUStride];
+  __shared__ int row_a[kUH], row_b[kUH], col_a[kUW], col_b[kUW];
+  __shared__ float row_f[kUH], col_f[kUW];
   const int64_t plane = blockIdx.z;
   const int y0 = blockIdx.y * kTileH, x0 = blockIdx.x * kTileW;
   const float* __restrict__ lr = a.x_lr + plane * a.h * a.w;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int cx = 4 * tx;  // first tile column of this thread
+  const int x = x0 + cx;
+  // The noise this thread blends, requested first so that its DRAM latency
+  // overlaps the upsampling below.
+  float4 nz[4];
+  if (VEC) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int y = y0 + ty + 8 * k;
+      nz[k] = (y < a.H && x + 3 < a.W)
+                  ? __ldcs(reinterpret_cast<const float4*>(a.noise +
+                                                           (plane * a.H + y) * (int64_t)a.W + x))
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
 
-  // u on the tile and its halo, at clamped high-res coordinates.
+  // Source taps of the tile's rows and columns (with the halo, clamped to
+  // the image), once per CTA.
+  for (int i = threadIdx.x; i < kUH + kUW; i += kThreads) {
+    if (i < kUH) {
+      taps(min(max(y0 - 1 + i, 0), a.H - 1), a.s, a.h, row_a[i], row_b[i], row_f[i]);
+    } else {
+      const int c = i - kUH;
+      taps(min(max(x0 - 1 + c, 0), a.W - 1), a.s, a.w, col_a[c], col_b[c], col_f[c]);
+    }
+  }
+  __syncthreads();
+  // u on the tile and its halo.
   for (int i = threadIdx.x; i < kUH * kUW; i += kThreads) {
     const int r = i / kUW, c = i - (i / kUW) * kUW;
-    const int y = min(max(y0 - 1 + r, 0), a.H - 1);
-    const int x = min(max(x0 - 1 + c, 0), a.W - 1);
-    int ya, yb, xa, xb;
-    float fy, fx;
-    taps(y, a.s, a.h, ya, yb, fy);
-    taps(x, a.s, a.w, xa, xb, fx);
-    const float* ra = lr + (int64_t)ya * a.w;
-    const float* rb = lr + (int64_t)yb * a.w;
+    const float fy = row_f[r], fx = col_f[c];
+    const int xa = col_a[c], xb = col_b[c];
+    const float* ra = lr + (int64_t)row_a[r] * a.w;
+    const float* rb = lr + (int64_t)row_b[r] * a.w;
     const float top = __ldg(ra + xa) * (1.f - fx) + __ldg(ra + xb) * fx;
     const float bot = __ldg(rb + xa) * (1.f - fx) + __ldg(rb + xb) * fx;
     u[r][c] = top * (1.f - fy) + bot * fy;
   }
   __syncthreads();
 
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int cx = 4 * tx;  // first tile column of this thread
   const float keep = 1.f + a.amount, t1 = 1.f - a.t;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -98,10 +121,9 @@ __global__ void __launch_bounds__(kThreads) warm_start_kernel(const WarmArgs a) 
       const float c = u[ry + 1][cx + 1 + j];
       res[j] = t1 * (keep * c - a.amount * b);
     }
-    const int x = x0 + cx;
     const int64_t off = (plane * a.H + y) * (int64_t)a.W + x;
     if (VEC && x + 3 < a.W) {
-      const float4 n = __ldcs(reinterpret_cast<const float4*>(a.noise + off));
+      const float4 n = nz[k];
       float4 o;
       o.x = fmaf(a.t, n.x, res[0]);
       o.y = fmaf(a.t, n.y, res[1]);

@@ -99,11 +99,14 @@ def test_attention_backward_sampled_4k():
     check(gq[:, rows], ref[0], bnd[0], "4K dq")
     check(gk[:, keys], ref[1], bnd[1], "4K dk")
     check(gv[:, keys], ref[2], bnd[2], "4K dv")
-    # identities of any softmax attention, all heads, every key
-    gq, gk, gv = joint_grads(grads, wl)
-    do = joint_f64(x, "do")
-    assert np.all(np.abs(gv.sum(1) - do.sum(1)) <= 2 * U * np.abs(gv).sum(1) + 1e-3)
-    assert np.all(np.abs(gk.sum(1)) <= 4 * U * np.abs(gk).sum(1) + 1e-3)
+    # identities of any softmax attention, all heads, every key (sums in fp64
+    # on the device)
+    tot = lambda a, b_: a.double().sum(1) + b_.double().sum(1)
+    mag = lambda a, b_: a.double().abs().sum(1) + b_.double().abs().sum(1)
+    dk_hr, dv_hr, dk_lr, dv_lr = grads[1], grads[2], grads[4], grads[5]
+    do_sum = tot(x["do_hr"].to(DEV), x["do_lr"].to(DEV))
+    assert bool(((tot(dv_hr, dv_lr) - do_sum).abs() <= 2 * U * mag(dv_hr, dv_lr) + 1e-3).all())
+    assert bool((tot(dk_hr, dk_lr).abs() <= 4 * U * mag(dk_hr, dk_lr) + 1e-3).all())
 
 
 SETS = [(ug.UG_HR_WINDOW_FIRST, O.HR_WINDOW_FIRST), (ug.UG_HR_RASTER, O.HR_RASTER),
