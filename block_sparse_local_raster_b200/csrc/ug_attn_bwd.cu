@@ -660,23 +660,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ++gphase;
       return r;
     };
+    // Per-query lse (log2 units) and D of a tile, one entry per thread;
+    // queries past the tensor get probability 0 and D = 0.  Loaded one tile
+    // of this warpgroup ahead, so the load latency is off the critical path.
+    auto load_stats = [&](int i, float& l, float& dd) {
+      l = __int_as_float(0x7f800000);
+      dd = 0.0f;
+      if (i < nq) {
+        const uint32_t e = P.qlist[kt.list_off + i];
+        const bool qlr = (e & kBlockLowres) != 0;
+        const int q = (int)(e & kBlockIndexMask) * kRowsPerTile + row;
+        if (q < (qlr ? P.L : P.N)) {
+          const int64_t ri = hbase + (qlr ? P.N : 0) + q;
+          l = P.lse[ri] * kLog2e;
+          dd = P.delta[ri];
+        }
+      }
+    };
+    float nx_lse, nx_dlt;
+    load_stats(g, nx_lse, nx_dlt);
     bool ok = true;
     for (int i = g; i < nq; i += 2) {
       const uint32_t e = P.qlist[kt.list_off + i];
       const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-      const bool qlr = (e & kBlockLowres) != 0;
       const int q0 = (int)(e & kBlockIndexMask) * kRowsPerTile;
-      const int nqt = qlr ? P.L : P.N;
-      // This tile's per-query lse (log2 units) and D, one entry per thread;
-      // queries past the tensor get probability 0 and D = 0.
       if (!(ok = group_sync())) break;  // the previous tile's readers are done
-      {
-        const int q = q0 + row;
-        const bool v = q < nqt;
-        const int64_t ri = hbase + (qlr ? P.N : 0) + q;
-        my_lse[row] = v ? P.lse[ri] * kLog2e : __int_as_float(0x7f800000);
-        my_dlt[row] = v ? P.delta[ri] : 0.0f;
-      }
+      my_lse[row] = nx_lse;
+      my_dlt[row] = nx_dlt;
+      load_stats(i + 2, nx_lse, nx_dlt);
       if (!(ok = group_sync())) break;
       if (!(ok = wait_warp(s_full(g), ph))) break;
       fence_after();

@@ -52,6 +52,10 @@ __device__ __forceinline__ void taps(int d, int s, int n, int& i0, int& i1, floa
 template <bool VEC>
 __global__ void __launch_bounds__(kThreads) warm_start_kernel(const WarmArgs a) {
   __shared__ float u[kUH][kUStride];
+  // The low-res samples the tile reads.  Tap indices grow with the output
+  // coordinate and span at most one more sample than the tile has rows
+  // (columns), which happens at s = 1.
+  __shared__ float patch[(kUH + 1) * (kUW + 1)];
   __shared__ int row_a[kUH], row_b[kUH], col_a[kUW], col_b[kUW];
   __shared__ float row_f[kUH], col_f[kUW];
   const int64_t plane = blockIdx.z;
@@ -85,15 +89,23 @@ __global__ void __launch_bounds__(kThreads) warm_start_kernel(const WarmArgs a) 
     }
   }
   __syncthreads();
+  // The low-res rectangle the taps reach, staged once with coalesced loads.
+  const int r0 = row_a[0], pr = row_b[kUH - 1] - r0 + 1;
+  const int c0 = col_a[0], pc = col_b[kUW - 1] - c0 + 1;
+  for (int i = threadIdx.x; i < pr * pc; i += kThreads) {
+    const int r = i / pc, c = i - (i / pc) * pc;
+    patch[i] = __ldg(lr + (int64_t)(r0 + r) * a.w + c0 + c);
+  }
+  __syncthreads();
   // u on the tile and its halo.
   for (int i = threadIdx.x; i < kUH * kUW; i += kThreads) {
     const int r = i / kUW, c = i - (i / kUW) * kUW;
     const float fy = row_f[r], fx = col_f[c];
-    const int xa = col_a[c], xb = col_b[c];
-    const float* ra = lr + (int64_t)row_a[r] * a.w;
-    const float* rb = lr + (int64_t)row_b[r] * a.w;
-    const float top = __ldg(ra + xa) * (1.f - fx) + __ldg(ra + xb) * fx;
-    const float bot = __ldg(rb + xa) * (1.f - fx) + __ldg(rb + xb) * fx;
+    const int xa = col_a[c] - c0, xb = col_b[c] - c0;
+    const float* ra = patch + (row_a[r] - r0) * pc;
+    const float* rb = patch + (row_b[r] - r0) * pc;
+    const float top = ra[xa] * (1.f - fx) + ra[xb] * fx;
+    const float bot = rb[xa] * (1.f - fx) + rb[xb] * fx;
     u[r][c] = top * (1.f - fy) + bot * fy;
   }
   __syncthreads();
