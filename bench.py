@@ -572,7 +572,10 @@ def run_backward(args, wl, world, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": wl.name, "useful_flop_per_backward": flops,
-                       "l2": "inputs larger than L2, no flush"},
+                       "l2": ("inputs larger than L2 (each high-res tensor %.0f MB), no flush"
+                              if d["q_hr"].numel() * 2 > L2_BYTES else
+                              "inputs smaller than L2 (%.0f MB per high-res tensor), no flush")
+                             % (d["q_hr"].numel() * 2 / 1e6)},
             "attn_bwd_ms": attn * 1e3, "attn_bwd_tflops": ach,
             "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops_sustained"],
                          "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops_sustained"],

@@ -147,24 +147,49 @@ __device__ __forceinline__ void mma_tmem_rows(uint32_t d, uint32_t a_tmem, uint3
 
 // Masks the row's scores where a high-res pair is invisible: `mine` is the
 // window of this thread's row (query in dq_kernel, key in dkv_kernel), the
-// 128 columns are the tokens c0 .. c0+127 of the other side.  Visibility
+// COLS columns are the tokens c0 .. c0+COLS-1 of the other side.  Visibility
 // changes only at window boundaries, so each window met is tested once.
+template <int COLS>
 __device__ __forceinline__ void mask_windows(float* s, int c0, int mine, const BwdParams& P) {
   const int my = mine / P.nwx, mx = mine - (mine / P.nwx) * P.nwx;
   int i0 = 0;
-  while (i0 < kKeysPerBlock) {
+  while (i0 < COLS) {
     const int c = c0 + i0;
     const int w = c / P.T;
-    const int run = min(kKeysPerBlock, (w + 1) * P.T - c0);
+    const int run = min(COLS, (w + 1) * P.T - c0);
     const int wy = w / P.nwx, wx = w - (w / P.nwx) * P.nwx;
     const bool vis = abs(wy - my) <= P.radius && abs(wx - mx) <= P.radius;
     const int lim = vis ? min(run, P.N - c0) : i0;  // columns [i0, lim) stay
 #pragma unroll
-    for (int i = 0; i < kKeysPerBlock; ++i)
+    for (int i = 0; i < COLS; ++i)
       if (i >= i0 && i < run && i >= lim) s[i] = kNegInf;
     i0 = run;
   }
 }
+
+// Bounded polling for an issue loop that tests several barriers: gives up
+// (records UG_ERR_TIMEOUT, raises the abort flag) after timeout_ns without
+// progress, or when the abort flag is up.
+struct PollTimer {
+  uint64_t last;
+  uint32_t spins;
+  __device__ PollTimer() : last(globaltimer()), spins(0) {}
+  __device__ bool step(bool progressed, volatile uint32_t* abort, int* err, int64_t timeout_ns) {
+    if (progressed) {
+      spins = 0;
+      last = globaltimer();
+      return true;
+    }
+    if ((++spins & 15u) != 0u) return true;
+    if (*abort) return false;
+    if ((int64_t)(globaltimer() - last) > timeout_ns) {
+      atomicCAS(err, 0, (int)UG_ERR_TIMEOUT);
+      *abort = 1u;
+      return false;
+    }
+    return true;
+  }
+};
 
 // ------------------------------------------------------------------ dQ
 
@@ -313,34 +338,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t tQ = tmem + 256u;
       const uint32_t sQ = sbase + Lay::kQ, sDO = sbase + Lay::kDO;
       auto kv_addr = [&](int it) { return sbase + Lay::kKV + slot(it) * kTile; };
+      // Issue each step as soon as its inputs are ready: S_j = Q K_j^T (needs
+      // K_j and buffer j&1 free, i.e. dQ_{j-2} issued), dP_j = dO V_j^T over S_j
+      // (needs V_j and the softmax done reading S_j), dQ += dS_j K_j (needs
+      // dS_j).  Steps of one kind go in block order; no barrier is tested
+      // more than one phase ahead.
       bool ok = wait1(q_full, 0);
-      for (int j = 0; j < 2 && j < nblk && ok; ++j) {
-        if (!(ok = wait1(kv_full(slot(2 * j)), phase(2 * j)))) break;
-        fence_after();
-        mma_rows<D>(tB[j], sQ, kv_addr(2 * j));  // S_j = Q K_j^T
-        mma_commit(s_full(j));
-      }
-      for (int j = 0; j < nblk && ok; ++j) {
-        const int bb = j & 1;
-        const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-        const int ik = 2 * j, iv = 2 * j + 1;
-        if (!(ok = wait1(kv_full(slot(iv)), phase(iv)))) break;
-        if (!(ok = wait1(s_free(bb), ph))) break;
-        fence_after();
-        mma_rows<D>(tB[bb], sDO, kv_addr(iv));  // dP_j = dO V_j^T, over S_j
-        mma_commit(dp_full(bb));
-        mma_commit(kv_empty(slot(iv)));
-        if (!(ok = wait1(ds_full(bb), ph))) break;
-        fence_after();
-        mma_tmem_rows<D>(tQ, tB[bb], kv_addr(ik), j > 0);  // dQ += dS_j K_j
-        mma_commit(kv_empty(slot(ik)));
-        if (j + 2 < nblk) {
-          const int ik2 = 2 * (j + 2);
-          if (!(ok = wait1(kv_full(slot(ik2)), phase(ik2)))) break;
+      int ns = 0, na = 0, nb = 0;  // next S, next dP, next dQ
+      PollTimer poll;
+      while (ok && nb < nblk) {
+        bool did = true;
+        if (nb < na && mbar_test(ds_full(nb & 1), (uint32_t)(nb >> 1) & 1u)) {
           fence_after();
-          mma_rows<D>(tB[bb], sQ, kv_addr(ik2));  // S_{j+2}
-          mma_commit(s_full(bb));
+          mma_tmem_rows<D>(tQ, tB[nb & 1], kv_addr(2 * nb), nb > 0);  // dQ += dS_j K_j
+          mma_commit(kv_empty(slot(2 * nb)));
+          ++nb;
+        } else if (na < ns && mbar_test(kv_full(slot(2 * na + 1)), phase(2 * na + 1)) &&
+                   mbar_test(s_free(na & 1), (uint32_t)(na >> 1) & 1u)) {
+          fence_after();
+          mma_rows<D>(tB[na & 1], sDO, kv_addr(2 * na + 1));  // dP_j = dO V_j^T, over S_j
+          mma_commit(dp_full(na & 1));
+          mma_commit(kv_empty(slot(2 * na + 1)));
+          ++na;
+        } else if (ns < nblk && ns <= nb + 1 && mbar_test(kv_full(slot(2 * ns)), phase(2 * ns))) {
+          fence_after();
+          mma_rows<D>(tB[ns & 1], sQ, kv_addr(2 * ns));  // S_j = Q K_j^T
+          mma_commit(s_full(ns & 1));
+          ++ns;
+        } else {
+          did = false;
         }
+        ok = poll.step(did, abort, err, timeout_ns);
       }
       if (ok) mma_commit(dq_done);
       mma_commit(drain);
@@ -364,28 +392,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t ph = (uint32_t)(j >> 1) & 1u;
       if (!(ok = wait_warp(s_full(g), ph))) break;
       fence_after();
-      float s[kKeysPerBlock];
-#pragma unroll
-      for (int c = 0; c < kKeysPerBlock / 32; ++c) tmem_ld32(tb + c * 32, s + c * 32);
-      tmem_ld_wait();
-      if (e & kBlockMasked) {
-        const int k0 = (int)(e & kBlockIndexMask) * kKeysPerBlock;
-        if (e & kBlockLowres) {
-#pragma unroll
-          for (int i = 0; i < kKeysPerBlock; ++i)
-            if (k0 + i >= P.L) s[i] = kNegInf;
-        } else {
-          mask_windows(s, k0, q_w, P);
-        }
-      }
-      // P = 2^(s * scale * log2e - lse2), kept as bf16 pairs for dS.
+      // P = 2^(s * scale * log2e - lse2), kept as bf16 pairs for dS; the
+      // scores are read in two halves of 64 keys to bound register use.
       uint32_t pk[kKeysPerBlock / 2];
       const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
       const float2 nl2 = make_float2(-lse2, -lse2);
 #pragma unroll
-      for (int i = 0; i < kKeysPerBlock; i += 2) {
-        const float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), sc2, nl2);
-        pk[i / 2] = pack_bf16(fast_exp2(x.x), fast_exp2(x.y));
+      for (int hf = 0; hf < 2; ++hf) {
+        float s[64];
+        tmem_ld32(tb + 64 * hf, s);
+        tmem_ld32(tb + 64 * hf + 32, s + 32);
+        tmem_ld_wait();
+        if (e & kBlockMasked) {
+          const int k0 = (int)(e & kBlockIndexMask) * kKeysPerBlock + 64 * hf;
+          if (e & kBlockLowres) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (k0 + i >= P.L) s[i] = kNegInf;
+          } else {
+            mask_windows<64>(s, k0, q_w, P);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          const float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), sc2, nl2);
+          pk[32 * hf + i / 2] = pack_bf16(fast_exp2(x.x), fast_exp2(x.y));
+        }
       }
       fence_before();
       mbar_arrive(s_free(g));  // S read: dP may overwrite the buffer
@@ -607,35 +639,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t tdV = tmem + 256u, tdK = tmem + 384u;
       const uint32_t sK = sbase + Lay::kK, sV = sbase + Lay::kV;
       auto ring_addr = [&](int it) { return sbase + Lay::kRingOff + slot(it) * kTile; };
+      // As in dq_kernel: S^T_i = K Q_i^T (needs Q_i and buffer i&1 free, i.e.
+      // dK_{i-2} issued), then dV += P^T_i dO_i and dP^T_i = V dO_i^T (need
+      // dO_i and P^T_i), then dK += dS^T_i Q_i (needs dS^T_i), each kind in
+      // tile order, issued as soon as ready.
       bool ok = wait1(kv_full, 0);
-      for (int i = 0; i < 2 && i < nq && ok; ++i) {
-        if (!(ok = wait1(ring_full(slot(2 * i)), phase(2 * i)))) break;
-        fence_after();
-        mma_rows<D>(tB[i], sK, ring_addr(2 * i));  // S^T_i = K Q_i^T
-        mma_commit(s_full(i));
-      }
-      for (int i = 0; i < nq && ok; ++i) {
-        const int bb = i & 1;
-        const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-        const int iq = 2 * i, ido = 2 * i + 1;
-        if (!(ok = wait1(ring_full(slot(ido)), phase(ido)))) break;
-        if (!(ok = wait1(p_full(bb), ph))) break;
-        fence_after();
-        mma_tmem_rows<D>(tdV, tB[bb], ring_addr(ido), i > 0);  // dV += P^T_i dO_i
-        mma_rows<D>(tB[bb], sV, ring_addr(ido));               // dP^T_i = V dO_i^T
-        mma_commit(dp_full(bb));
-        mma_commit(ring_empty(slot(ido)));
-        if (!(ok = wait1(ds_full(bb), ph))) break;
-        fence_after();
-        mma_tmem_rows<D>(tdK, tB[bb], ring_addr(iq), i > 0);  // dK += dS^T_i Q_i
-        mma_commit(ring_empty(slot(iq)));
-        if (i + 2 < nq) {
-          const int iq2 = 2 * (i + 2);
-          if (!(ok = wait1(ring_full(slot(iq2)), phase(iq2)))) break;
+      int ns = 0, na = 0, nb = 0;
+      PollTimer poll;
+      while (ok && nb < nq) {
+        bool did = true;
+        if (nb < na && mbar_test(ds_full(nb & 1), (uint32_t)(nb >> 1) & 1u)) {
           fence_after();
-          mma_rows<D>(tB[bb], sK, ring_addr(iq2));  // S^T_{i+2}
-          mma_commit(s_full(bb));
+          mma_tmem_rows<D>(tdK, tB[nb & 1], ring_addr(2 * nb), nb > 0);  // dK += dS^T_i Q_i
+          mma_commit(ring_empty(slot(2 * nb)));
+          ++nb;
+        } else if (na < ns && mbar_test(ring_full(slot(2 * na + 1)), phase(2 * na + 1)) &&
+                   mbar_test(p_full(na & 1), (uint32_t)(na >> 1) & 1u)) {
+          fence_after();
+          mma_tmem_rows<D>(tdV, tB[na & 1], ring_addr(2 * na + 1), na > 0);  // dV += P^T_i dO_i
+          mma_rows<D>(tB[na & 1], sV, ring_addr(2 * na + 1));  // dP^T_i = V dO_i^T
+          mma_commit(dp_full(na & 1));
+          mma_commit(ring_empty(slot(2 * na + 1)));
+          ++na;
+        } else if (ns < nq && ns <= nb + 1 && mbar_test(ring_full(slot(2 * ns)), phase(2 * ns))) {
+          fence_after();
+          mma_rows<D>(tB[ns & 1], sK, ring_addr(2 * ns));  // S^T_i = K Q_i^T
+          mma_commit(s_full(ns & 1));
+          ++ns;
+        } else {
+          did = false;
         }
+        ok = poll.step(did, abort, err, timeout_ns);
       }
       if (ok) mma_commit(acc_done);
       mma_commit(drain);
@@ -691,21 +725,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!(ok = group_sync())) break;
       if (!(ok = wait_warp(s_full(g), ph))) break;
       fence_after();
-      float s[kRowsPerTile];
-#pragma unroll
-      for (int c = 0; c < kRowsPerTile / 32; ++c) tmem_ld32(tb + c * 32, s + c * 32);
-      tmem_ld_wait();
-      if (e & kBlockMasked) mask_windows(s, q0, k_w, P);
+      // P^T in two halves of 64 queries (bounded register use); half h
+      // writes its 32 bf16-pair columns over S^T columns it has just read.
       uint32_t pk[kRowsPerTile / 2];
       const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
 #pragma unroll
-      for (int c = 0; c < kRowsPerTile; c += 2) {
-        const float2 l2 = *reinterpret_cast<const float2*>(my_lse + c);
-        const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, make_float2(-l2.x, -l2.y));
-        pk[c / 2] = pack_bf16(fast_exp2(x.x), fast_exp2(x.y));
+      for (int hf = 0; hf < 2; ++hf) {
+        float s[64];
+        tmem_ld32(tb + 64 * hf, s);
+        tmem_ld32(tb + 64 * hf + 32, s + 32);
+        tmem_ld_wait();
+        if (e & kBlockMasked) mask_windows<64>(s, q0 + 64 * hf, k_w, P);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float2 l2 = *reinterpret_cast<const float2*>(my_lse + 64 * hf + c);
+          const float2 x =
+              __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, make_float2(-l2.x, -l2.y));
+          pk[32 * hf + c / 2] = pack_bf16(fast_exp2(x.x), fast_exp2(x.y));
+        }
+        tmem_st32u(tb + 32 * hf, pk + 32 * hf);
       }
-      tmem_st32u(tb, pk);
-      tmem_st32u(tb + 32, pk + 32);
       tmem_st_wait();
       fence_before();
       mbar_arrive(p_full(g));  // P^T in TMEM: dV += P^T dO, then dP^T over it
