@@ -154,15 +154,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def attn_source_hash() -> str:
+    """sha256 (16 hex digits) over the forward attention kernel's sources."""
+    csrc = os.path.join(ROOT, "block_sparse_local_raster_b200", "csrc")
+    hs = hashlib.sha256()
+    for f in ("ug_attn.cu", "ug_tc.cuh"):
+        hs.update(open(os.path.join(csrc, f), "rb").read())
+    return hs.hexdigest()[:16]
+
+
 def attn_traffic_bytes(config: str):
     """DRAM bytes per attention launch from the committed ncu summary, or None
     if the kernel source changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "attention_dram_traffic.json")
-    src = os.path.join(ROOT, "block_sparse_local_raster_b200", "csrc", "ug_attn.cu")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    h = attn_source_hash()
     e = d.get(config)
     if not e or e.get("source_sha256_16") != h:
         return None
