@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = (warp & 3) * 32 + lane;    // TMEM lane = query row of the tile
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tb = tmem + lane_base + (g ? 128u : 0u);
+    const uint32_t tp = tmem + lane_base + 384u + (g ? 64u : 0u);  // parked P (bf16 pairs)
     const int tok = q0 + row;
     const bool valid = tok < ntok;
     const int64_t ridx = ((int64_t)b * P.heads + head) * (P.N + P.L) + (qt.lowres ? P.N : 0) + tok;
@@ -392,13 +393,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t ph = (uint32_t)(j >> 1) & 1u;
       if (!(ok = wait_warp(s_full(g), ph))) break;
       fence_after();
-      // P = 2^(s * scale * log2e - lse2), kept as bf16 pairs for dS; the
-      // scores are read in two halves of 64 keys to bound register use.
-      uint32_t pk[kKeysPerBlock / 2];
+      // P = 2^(s * scale * log2e - lse2) as bf16 pairs, parked in this
+      // warpgroup's 64 columns of the last TMEM quarter until dS needs it;
+      // the scores are read in two halves of 64 keys.
       const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
       const float2 nl2 = make_float2(-lse2, -lse2);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
         float s[64];
         tmem_ld32(tb + 64 * hf, s);
         tmem_ld32(tb + 64 * hf + 32, s + 32);
@@ -416,9 +418,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int i = 0; i < 64; i += 2) {
           const float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), sc2, nl2);
-          pk[32 * hf + i / 2] = pack_bf16(fast_exp2(x.x), fast_exp2(x.y));
+          pk[i / 2] = pack_bf16(fast_exp2(x.x), fast_exp2(x.y));
         }
+        tmem_st32u(tp + 32 * hf, pk);
       }
+      tmem_st_wait();
       fence_before();
       mbar_arrive(s_free(g));  // S read: dP may overwrite the buffer
       if (!(ok = wait_warp(dp_full(g), ph))) break;
@@ -428,12 +432,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int c = 0; c < kKeysPerBlock / 32; ++c) {
         float dp[32];
+        float pf[16];
         tmem_ld32(tb + c * 32, dp);
+        tmem_ld16(tp + c * 16, pf);
         tmem_ld_wait();
+        const uint32_t* pk = reinterpret_cast<const uint32_t*>(pf);
         uint32_t ds[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float2 p = unpack_bf16(pk[c * 16 + i / 2]);
+          const float2 p = unpack_bf16(pk[i / 2]);
           ds[i / 2] = pack_bf16(p.x * (dp[i] - dlt), p.y * (dp[i + 1] - dlt));
         }
         tmem_st16u(tb + c * 16, ds);
