@@ -595,11 +595,37 @@ def run_backward(args, wl, world, rank, local):
                     "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in grads)},
             "gpu_launches": launches * args.steps, "clocks": clk,
         }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = backward_cpu_baseline(wl, x)
         print(json.dumps(line), flush=True)
     plan.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def backward_cpu_baseline(wl, x):
+    """The oracle's attention backward, as it stands, on a bounded sample:
+    dQ of 16 high-res and 4 global query rows of head 0 (each row's full
+    softmax over every key it sees), rotated q/k recomputed.  Useful FLOPs of
+    the sample: 2.5 x 4 d x (visible keys of the sampled rows)."""
+    from oracle import hier_local_attn as O
+    g = O.Geometry.from_dict(dict(wl.geom_dict(), heads=1))
+    bits = {k: v[:, :, :1].contiguous().view(torch.int16).numpy().view(np.uint16)
+            for k, v in x.items()}
+    rng = np.random.default_rng(0)
+    rows = np.sort(np.concatenate([rng.choice(g.N, 16, replace=False),
+                                   g.N + rng.choice(g.L, 4, replace=False) if g.L else []])
+                   ).astype(np.int64)
+    vis = int(sum(O.visibility(g, O.HR_RASTER, rows[i:i + 1]).sum() for i in range(rows.size)))
+    c0 = time.perf_counter()
+    O.layer_backward(bits, bits, g, rows=rows, keys=np.zeros(0, dtype=np.int64))
+    cdt = time.perf_counter() - c0
+    flops = 2.5 * 4 * g.head_dim * vis
+    return {"value": flops / cdt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+            "kind": "oracle",
+            "sample": (f"dq of {rows.size} query rows x 1 head of the {wl.name} layer backward "
+                       f"(RoPE of every key included), fp64 numpy, {cdt:.1f} s")}
 
 
 def run_warm_start(args, world, rank, local):
