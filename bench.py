@@ -2,9 +2,12 @@
 """Benchmark of one hierarchical-local-attention layer on B200.
 
 A step is one pass of the whole layer over one batch of synthetic raster-order
-inputs already resident in HBM: window-first permute of q, k, v with the RoPE
-of q and k applied in the same pass (3 launches), RoPE of the low-res q and k
-(2), block-sparse attention (1), unpermute of the output (1).  The metric is useful attention TFLOP/s
+inputs already resident in HBM: window-first permute of q and k with their RoPE
+applied in the same pass (2 launches), RoPE of the global q and k (2), the
+block-sparse attention (1).  Where 128-key tiles are whole window rows (2K, 4K,
+8K, 4K-CFG) the attention reads v and writes o in raster order itself;
+elsewhere v is permuted first and o unpermuted after (2 more launches).  The
+metric is useful attention TFLOP/s
 (4 * head_dim FLOPs per visible query-key pair per head) over the step, with
 ms per layer; the attention kernel alone is also timed and set against the
 measured bf16 tensor peak.
@@ -284,22 +287,34 @@ def run_ug(args, wl, world, rank, local):
         if st != ug.UG_OK:
             raise ug.UgError(st, what)
 
+    # where 128-key tiles are whole window rows the attention reads v and
+    # writes o in raster order (no permute of v, no unpermute of o)
+    T = wl.win_h * wl.win_w
+    vo_raster = 128 % wl.win_w == 0 and T % 128 == 0
+
     def step(ev=None):
         chk(plan.permute_rope_window_first(d["q_hr"], ws_q), "permute+rope q")
         chk(plan.permute_rope_window_first(d["k_hr"], ws_k), "permute+rope k")
-        chk(plan.permute_window_first(d["v_hr"], ws_v), "permute v")
+        if not vo_raster:
+            chk(plan.permute_window_first(d["v_hr"], ws_v), "permute v")
         if L:
             chk(plan.rope_2d(d["q_lr"], ws_ql, ug.UG_LR), "rope q_lr")
             chk(plan.rope_2d(d["k_lr"], ws_kl, ug.UG_LR), "rope k_lr")
         if ev is not None:
             ev[0].record(stream)
-        chk(plan.hier_local_attn_fwd(ws_q, ws_k, ws_v, ws_ql, ws_kl, d["v_lr"] if L else None,
-                                     ws_o, o_lr, lse), "attention")
+        if vo_raster:
+            chk(plan.hier_local_attn_fwd_vo_raster(ws_q, ws_k, d["v_hr"], ws_ql, ws_kl,
+                                                   d["v_lr"] if L else None, o_hr, o_lr, lse),
+                "attention")
+        else:
+            chk(plan.hier_local_attn_fwd(ws_q, ws_k, ws_v, ws_ql, ws_kl,
+                                         d["v_lr"] if L else None, ws_o, o_lr, lse), "attention")
         if ev is not None:
             ev[1].record(stream)
-        chk(plan.unpermute(ws_o, o_hr), "unpermute")
+        if not vo_raster:
+            chk(plan.unpermute(ws_o, o_hr), "unpermute")
 
-    launches_per_step = 3 + (2 if L else 0) + 1 + 1
+    launches_per_step = 2 + (2 if L else 0) + 1 + (0 if vo_raster else 2)
     flops = useful_flops(wl)
 
     for _ in range(args.warmup):

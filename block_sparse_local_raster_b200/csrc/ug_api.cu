@@ -206,9 +206,13 @@ int ug_rope_2d(const ug_plan* p, const void* x, void* y, int token_set, void* s)
   return launch_rope(p, x, y, token_set, as_stream(s));
 }
 
-int ug_hier_local_attn_fwd(const ug_plan* p, const void* q_hr, const void* k_hr,
-                           const void* v_hr, const void* q_lr, const void* k_lr,
-                           const void* v_lr, void* o_hr, void* o_lr, float* lse, void* s) {
+}  // extern "C"
+
+namespace {
+
+int attn_fwd_checked(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+                     const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
+                     void* o_lr, float* lse, bool vo_raster, void* s) {
   if (!p || !q_hr || !k_hr || !v_hr || !o_hr) return UG_ERR_INVALID_ARG;
   if (p->L > 0 && (!q_lr || !k_lr || !v_lr || !o_lr)) return UG_ERR_INVALID_ARG;
   if (p->g.head_dim != 64 && p->g.head_dim != 128) return UG_ERR_UNSUPPORTED;
@@ -228,9 +232,29 @@ int ug_hier_local_attn_fwd(const ug_plan* p, const void* q_hr, const void* k_hr,
   if (overlap(o_hr, nh, o_lr, nl) || overlap(o_hr, nh, lse, nlse) || overlap(o_lr, nl, lse, nlse))
     return UG_ERR_ALIAS;
   return launch_attention(p, q_hr, k_hr, v_hr, p->L ? q_lr : nullptr, p->L ? k_lr : nullptr,
-                          p->L ? v_lr : nullptr, o_hr, p->L ? o_lr : nullptr, lse,
+                          p->L ? v_lr : nullptr, o_hr, p->L ? o_lr : nullptr, lse, vo_raster,
                           as_stream(s));
 }
+
+}  // namespace
+
+extern "C" {
+
+int ug_hier_local_attn_fwd(const ug_plan* p, const void* q_hr, const void* k_hr,
+                           const void* v_hr, const void* q_lr, const void* k_lr,
+                           const void* v_lr, void* o_hr, void* o_lr, float* lse, void* s) {
+  return attn_fwd_checked(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, false, s);
+}
+
+int ug_hier_local_attn_fwd_vo_raster(const ug_plan* p, const void* q_hr, const void* k_hr,
+                                     const void* v_hr_raster, const void* q_lr, const void* k_lr,
+                                     const void* v_lr, void* o_hr_raster, void* o_lr, float* lse,
+                                     void* s) {
+  if (p && !vo_raster_supported(p->g)) return UG_ERR_UNSUPPORTED;
+  return attn_fwd_checked(p, q_hr, k_hr, v_hr_raster, q_lr, k_lr, v_lr, o_hr_raster, o_lr, lse,
+                          true, s);
+}
+
 
 int64_t ug_layer_workspace_bytes(const ug_plan* p) {
   if (!p) return -1;
@@ -266,11 +290,16 @@ int ug_layer_fwd(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   int st;
   if ((st = ug_permute_rope_window_first(p, q_hr, q_wf, s)) != UG_OK) return st;
   if ((st = ug_permute_rope_window_first(p, k_hr, k_wf, s)) != UG_OK) return st;
-  if ((st = ug_permute_window_first(p, v_hr, v_wf, s)) != UG_OK) return st;
   if (p->L > 0) {
     if ((st = ug_rope_2d(p, q_lr, q_lr_r, UG_LR, s)) != UG_OK) return st;
     if ((st = ug_rope_2d(p, k_lr, k_lr_r, UG_LR, s)) != UG_OK) return st;
   }
+  // Where 128-key tiles are whole window rows, the attention reads v and
+  // writes o in raster order itself: no permute of v, no unpermute of o.
+  if (vo_raster_supported(p->g))
+    return ug_hier_local_attn_fwd_vo_raster(p, q_wf, k_wf, v_hr, q_lr_r, k_lr_r, v_lr, o_hr,
+                                            o_lr, lse, s);
+  if ((st = ug_permute_window_first(p, v_hr, v_wf, s)) != UG_OK) return st;
   if ((st = ug_hier_local_attn_fwd(p, q_wf, k_wf, v_wf, q_lr_r, k_lr_r, v_lr, o_wf, o_lr, lse,
                                    s)) != UG_OK)
     return st;

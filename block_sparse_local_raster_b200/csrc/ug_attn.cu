@@ -81,7 +81,19 @@ struct AttnParams {
   int64_t timeout_ns;
   int32_t N, L, T, nwx, radius, heads;
   float scale_log2;  // softmax scale * log2(e)
+  // Raster-order high-res V (read through a 5-D tensor map, one 128-key
+  // tile = 128 / win_w whole rows of one window) and raster-order o_hr.
+  int32_t vo_raster;
+  int32_t grid_w, win_h, win_w;
 };
+
+// Raster index of the high-res token at window-first position p.
+__device__ __forceinline__ int raster_of(int p, const AttnParams& P) {
+  const int w = p / P.T, l = p - (p / P.T) * P.T;
+  const int wy = w / P.nwx, wx = w - (w / P.nwx) * P.nwx;
+  const int ly = l / P.win_w, lx = l - (l / P.win_w) * P.win_w;
+  return (wy * P.win_h + ly) * P.grid_w + wx * P.win_w + lx;
+}
 
 // ---------------------------------------------------------------- the kernel
 
@@ -198,9 +210,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_expect_tx(kv_full(s), Lay::kTileBytes);
-          for (int r = 0; r < kRegions; ++r)
-            tma_load_4d(sbase + Lay::kKV + s * Lay::kTileBytes + r * kKeysPerBlock * 128, m,
-                        r * 64, head, k0, b, kv_full(s));
+          if (kv == 1 && !lr && P.vo_raster) {
+            // the block's keys are 128 / win_w whole rows of one window
+            const int w = k0 / P.T, ly0 = (k0 - (k0 / P.T) * P.T) / P.win_w;
+            const int wy = w / P.nwx, wx = w - (w / P.nwx) * P.nwx;
+            for (int r = 0; r < kRegions; ++r)
+              tma_load_5d(sbase + Lay::kKV + s * Lay::kTileBytes + r * kKeysPerBlock * 128, m,
+                          r * 64, head, wx * P.win_w, wy * P.win_h + ly0, b, kv_full(s));
+          } else {
+            for (int r = 0; r < kRegions; ++r)
+              tma_load_4d(sbase + Lay::kKV + s * Lay::kTileBytes + r * kKeysPerBlock * 128, m,
+                          r * 64, head, k0, b, kv_full(s));
+          }
         }
       }
       // Loads still in flight land before the CTA may exit.  The last
@@ -382,8 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ntok = qt.lowres ? P.L : P.N;
       const bool valid = tok < ntok;
       const float inv_l = 1.0f / l;
+      const int orow = (!qt.lowres && P.vo_raster && valid) ? raster_of(tok, P) : tok;
       __nv_bfloat16* dst = (qt.lowres ? P.o_lr : P.o_hr) +
-                           (((int64_t)b * ntok + tok) * P.heads + head) * D;
+                           (((int64_t)b * ntok + orow) * P.heads + head) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
@@ -420,15 +442,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 int launch_d(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
              const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr, void* o_lr,
-             float* lse, cudaStream_t st) {
+             float* lse, bool vo_raster, cudaStream_t st) {
   const int64_t B = p->g.batch;
   const int H = p->g.heads;
   CUtensorMap m[6];
   const void* lrs[3] = {q_lr ? q_lr : q_hr, k_lr ? k_lr : k_hr, v_lr ? v_lr : v_hr};
   const int64_t nl = p->L > 0 ? p->L : p->N;
-  if (!make_map(&m[0], q_hr, B, p->N, H, D) || !make_map(&m[1], k_hr, B, p->N, H, D) ||
-      !make_map(&m[2], v_hr, B, p->N, H, D) || !make_map(&m[3], lrs[0], B, nl, H, D) ||
-      !make_map(&m[4], lrs[1], B, nl, H, D) || !make_map(&m[5], lrs[2], B, nl, H, D))
+  const bool vmap = vo_raster ? make_map_raster(&m[2], v_hr, B, p->g.grid_h, p->g.grid_w, H, D,
+                                                p->g.win_w)
+                              : make_map(&m[2], v_hr, B, p->N, H, D);
+  if (!make_map(&m[0], q_hr, B, p->N, H, D) || !make_map(&m[1], k_hr, B, p->N, H, D) || !vmap ||
+      !make_map(&m[3], lrs[0], B, nl, H, D) || !make_map(&m[4], lrs[1], B, nl, H, D) ||
+      !make_map(&m[5], lrs[2], B, nl, H, D))
     return UG_ERR_CUDA;
   AttnParams P;
   P.qtiles = p->d_qtiles;
@@ -445,6 +470,10 @@ int launch_d(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v
   P.radius = p->g.radius;
   P.heads = H;
   P.scale_log2 = p->scale * 1.4426950408889634f;
+  P.vo_raster = vo_raster ? 1 : 0;
+  P.grid_w = p->g.grid_w;
+  P.win_h = p->g.win_h;
+  P.win_w = p->g.win_w;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(hier_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -462,12 +491,17 @@ int launch_d(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v
 
 int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                      const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
-                     void* o_lr, float* lse, cudaStream_t st) {
+                     void* o_lr, float* lse, bool vo_raster, cudaStream_t st) {
   if (p->g.head_dim == 128)
-    return launch_d<128>(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, st);
+    return launch_d<128>(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, vo_raster, st);
   if (p->g.head_dim == 64)
-    return launch_d<64>(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, st);
+    return launch_d<64>(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, vo_raster, st);
   return UG_ERR_UNSUPPORTED;
+}
+
+bool vo_raster_supported(const ug_geom& g) {
+  const int64_t T = (int64_t)g.win_h * g.win_w;
+  return g.win_w <= kRowsPerTile && kRowsPerTile % g.win_w == 0 && T % kRowsPerTile == 0;
 }
 
 }  // namespace ug

@@ -119,7 +119,10 @@ int launch_warm_start(const ug_warm_start_params* p, const float* x_lr, const fl
                       float* out, cudaStream_t s);
 int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                      const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
-                     void* o_lr, float* lse, cudaStream_t s);
+                     void* o_lr, float* lse, bool vo_raster, cudaStream_t s);
+// Whether a 128-key tile is always 128 / win_w whole rows of one window, so
+// that raster-order V can be read tile by tile.
+bool vo_raster_supported(const ug_geom& g);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

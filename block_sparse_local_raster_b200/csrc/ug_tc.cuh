@@ -81,6 +81,16 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int32_t c0,
+                                            int32_t c1, int32_t c2, int32_t c3, int32_t c4,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -255,6 +265,24 @@ EncodeTiledFn get_encode() {
 }
 
 // [B, n_tok, heads, D] bf16 -> box of 64 channels x 1 head x 128 tokens.
+// [B, grid_h, grid_w, heads, D] bf16 (a raster-order high-res tensor) ->
+// box of 64 channels x 1 head x win_w columns x (128 / win_w) rows: one
+// 128-token window-first tile, rows of the window in order.
+bool make_map_raster(CUtensorMap* m, const void* base, int64_t B, int grid_h, int grid_w,
+                     int heads, int D, int win_w) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)grid_w,
+                              (cuuint64_t)grid_h, (cuuint64_t)B};
+  const cuuint64_t row = (cuuint64_t)heads * D * 2;
+  const cuuint64_t strides[4] = {(cuuint64_t)D * 2, row, row * grid_w, row * grid_w * grid_h};
+  const cuuint32_t box[5] = {64, 1, (cuuint32_t)win_w, (cuuint32_t)(kRowsPerTile / win_w), 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map(CUtensorMap* m, const void* base, int64_t B, int64_t n_tok, int heads, int D) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;

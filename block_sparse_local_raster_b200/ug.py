@@ -35,7 +35,7 @@ EXPORTS = (
     "ug_geom_validate", "ug_index_map_sizes", "ug_build_index_maps", "ug_visible_pairs",
     "ug_status_string", "ug_plan_create", "ug_plan_destroy", "ug_get_index_maps",
     "ug_permute_window_first", "ug_permute_rope_window_first", "ug_unpermute", "ug_rope_2d",
-    "ug_hier_local_attn_fwd",
+    "ug_hier_local_attn_fwd", "ug_hier_local_attn_fwd_vo_raster",
     "ug_layer_workspace_bytes", "ug_layer_fwd", "ug_layer_fwd_static_scratch",
     "ug_plan_set_wait_timeout", "ug_check_error", "ug_warm_start",
     "ug_rope_2d_bwd", "ug_unpermute_rope_bwd", "ug_attn_bwd_workspace_bytes",
@@ -102,6 +102,7 @@ def lib() -> ctypes.CDLL:
         "ug_unpermute": (I32, [P, P, P, P]),
         "ug_rope_2d": (I32, [P, P, P, I32, P]),
         "ug_hier_local_attn_fwd": (I32, [P, P, P, P, P, P, P, P, P, P, P]),
+        "ug_hier_local_attn_fwd_vo_raster": (I32, [P, P, P, P, P, P, P, P, P, P, P]),
         "ug_layer_workspace_bytes": (I64, [P]),
         "ug_layer_fwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I64, P]),
         "ug_layer_fwd_static_scratch": (I32, [P, P, P, P, P, P, P, P, P, P, P]),
@@ -232,6 +233,12 @@ class Plan:
         return lib().ug_hier_local_attn_fwd(
             self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr), _ptr(q_lr), _ptr(k_lr), _ptr(v_lr),
             _ptr(o_hr), _ptr(o_lr), _ptr(lse), _stream(stream))
+
+    def hier_local_attn_fwd_vo_raster(self, q_hr, k_hr, v_hr_raster, q_lr, k_lr, v_lr,
+                                      o_hr_raster, o_lr, lse=None, stream=None) -> int:
+        return lib().ug_hier_local_attn_fwd_vo_raster(
+            self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr_raster), _ptr(q_lr), _ptr(k_lr),
+            _ptr(v_lr), _ptr(o_hr_raster), _ptr(o_lr), _ptr(lse), _stream(stream))
 
     def layer_fwd(self, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, workspace,
                   stream=None) -> int:

@@ -194,6 +194,20 @@ int ug_hier_local_attn_fwd(const ug_plan* plan, const void* q_hr, const void* k_
                            const void* v_hr, const void* q_lr, const void* k_lr,
                            const void* v_lr, void* o_hr, void* o_lr, float* lse, void* stream);
 
+/* Step 3 reading v and writing o in raster order, which removes the
+ * permutation of v and the unpermutation of o from the layer.  The same
+ * attention as ug_hier_local_attn_fwd with q_hr, k_hr window-first (rotated)
+ * but v_hr_raster [B, N, h, d] in raster order and o_hr_raster written in
+ * raster order; the global tensors and lse (high-res rows window-first) as
+ * there.  Each 128-key tile of V is read as 128 / win_w whole rows of one
+ * window, so the call needs win_w dividing 128 and 128 dividing
+ * win_h * win_w (UG_ERR_UNSUPPORTED otherwise; the 2K, 4K, 8K and 4K-CFG
+ * geometries qualify).  ug_layer_fwd uses it where it applies. */
+int ug_hier_local_attn_fwd_vo_raster(const ug_plan* plan, const void* q_hr, const void* k_hr,
+                                     const void* v_hr_raster, const void* q_lr, const void* k_lr,
+                                     const void* v_lr, void* o_hr_raster, void* o_lr, float* lse,
+                                     void* stream);
+
 /* ---- the whole layer ------------------------------------------------------ */
 
 /* Bytes of device scratch that ug_layer_fwd needs (window-first copies of the
@@ -203,8 +217,10 @@ int64_t ug_layer_workspace_bytes(const ug_plan* plan);
 /* Steps 1-4 in order on raster-order inputs: window-first permute of
  * q_hr, k_hr, v_hr (q and k with their RoPE applied in the same pass, as
  * ug_permute_rope_window_first); RoPE of the global q and k (rho-scaled
- * low-res positions, text rows unchanged); attention; unpermute of the high-res output into o_hr (raster
- * order).  q/k/v are not modified.  lse as in
+ * low-res positions, text rows unchanged); attention; unpermute of the
+ * high-res output into o_hr (raster order).  Where
+ * ug_hier_local_attn_fwd_vo_raster applies, the attention reads v_hr and
+ * writes o_hr in raster order itself instead.  q/k/v are not modified.  lse as in
  * ug_hier_local_attn_fwd (its high-res rows stay in window-first order).
  * workspace: caller-owned device scratch of at least
  * ug_layer_workspace_bytes(plan) bytes, 256-byte aligned; the call uses it

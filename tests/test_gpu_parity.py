@@ -172,6 +172,39 @@ def test_attention_sampled_rows(name):
     check_rows(wl, g, o_hr, o_lr, lse, ref_o, ref_lse, rows, vs)
 
 
+@pytest.mark.parametrize("name", SMALL + BIG)
+def test_attention_raster_v_and_o_equal_the_permuted_path(name):
+    """ug_hier_local_attn_fwd_vo_raster (v read, o written in raster order)
+    gives bit for bit the window-first attention's output, unpermuted, and
+    the same lse; geometries whose 128-key tiles are not whole window rows
+    are refused."""
+    wl = workloads.get(name)
+    p = plan(wl)
+    x = attn_inputs(wl, 320)
+    d = {k: v.to(DEV) for k, v in x.items() if k != "head_scale"}
+    has_lr = wl.n_lr > 0
+    lr = lambda n: d[n] if has_lr else None
+    T = wl.win_h * wl.win_w
+    supported = 128 % wl.win_w == 0 and T % 128 == 0
+    o_r = torch.empty_like(d["q_hr"])
+    o_lr = torch.empty_like(d["q_lr"]) if has_lr else None
+    lse = torch.empty((wl.batch, wl.heads, wl.n_hr + wl.n_lr), dtype=torch.float32, device=DEV)
+    v_raster = ug.unpermute(p, d["v_hr"])  # the same values in raster order
+    st = p.hier_local_attn_fwd_vo_raster(d["q_hr"], d["k_hr"], v_raster, lr("q_lr"), lr("k_lr"),
+                                         lr("v_lr"), o_r, o_lr, lse)
+    if not supported:
+        assert st == ug.UG_ERR_UNSUPPORTED
+        return
+    assert st == ug.UG_OK
+    o_hr, o_lr2, lse2 = run_attn(p, x)
+    torch.cuda.synchronize()
+    assert p.check_error() == ug.UG_OK
+    assert torch.equal(o_r, ug.unpermute(p, o_hr))
+    assert torch.equal(lse, lse2)
+    if has_lr:
+        assert torch.equal(o_lr, o_lr2)
+
+
 # ----------------------------------------------------------------- whole layer
 
 @pytest.mark.parametrize("name", SMALL + BIG)
