@@ -8,12 +8,15 @@
 //         direction with edges replicated (unsharp mask);
 //   out = (1 - t) * x0 + t * noise.
 //
-// HBM-bound: per high-res pixel one fp32 noise read and one fp32 write; the
-// low-res image (1/s^2 of that) is read through L1.  A CTA owns a 32 x 128
-// output tile of one plane: it evaluates u on the tile plus a one-pixel halo
-// into shared memory (rows and columns clamped at the image border, which is
-// the edge replication of the blur), then each thread blurs, sharpens and
-// blends 4 x 4 pixels, streaming noise in and the result out as float4.
+// Per high-res pixel one fp32 noise read and one fp32 write; the low-res
+// image (1/s^2 of that) is read through L1.  Each thread streams 4 adjacent
+// columns down a strip of kRows rows with everything in registers:
+// the source taps of its 6 columns (the 4 plus one on each side for the
+// blur), the two low-res rows it interpolates between (horizontally
+// interpolated at those 6 columns), and a rolling window of three upsampled
+// rows.  Its noise is requested before any arithmetic.  No shared memory and
+// no barrier: every warp streams on its own.  Clamping the rows and columns
+// of u at the image border is the blur's edge replication.
 #include <cstdint>
 
 #include "ug_internal.h"
@@ -21,12 +24,8 @@
 namespace ug {
 namespace {
 
-constexpr int kTileH = 32;
-constexpr int kTileW = 128;
-constexpr int kThreads = 256;  // 32 x 8: a thread owns 4 columns x 4 rows
-constexpr int kUH = kTileH + 2;
-constexpr int kUW = kTileW + 2;
-constexpr int kUStride = kUW + 2;
+constexpr int kThreads = 128;
+constexpr int kRows = 4;  // output rows per thread
 
 struct WarmArgs {
   const float* x_lr;
@@ -35,117 +34,152 @@ struct WarmArgs {
   int32_t h, w;     // low-res size
   int32_t H, W;     // high-res size
   int32_t s;        // upsampling factor
+  int32_t groups;   // ceil(W / 4) column groups per row
+  int32_t strips;   // ceil(H / kRows) row strips per plane
+  int64_t threads;  // planes * strips * groups
   float amount, t;
 };
 
-// Source coordinate of high-res index d along an axis of n low-res samples:
-// (d + 0.5) / s - 0.5 = (2d + 1 - s) / (2s).  The integer part and the
-// fraction are taken from the exact integer numerator.
-__device__ __forceinline__ void taps(int d, int s, int n, int& i0, int& i1, float& f) {
-  const int num = 2 * d + 1 - s, den = 2 * s;
-  const int fl = num >= 0 ? num / den : -((-num + den - 1) / den);
-  f = (float)(num - fl * den) / (float)den;
-  i0 = min(max(fl, 0), n - 1);
-  i1 = min(max(fl + 1, 0), n - 1);
-}
-
 template <bool VEC>
 __global__ void __launch_bounds__(kThreads) warm_start_kernel(const WarmArgs a) {
-  __shared__ float u[kUH][kUStride];
-  // The low-res samples the tile reads.  Tap indices grow with the output
-  // coordinate and span at most one more sample than the tile has rows
-  // (columns), which happens at s = 1.
-  __shared__ float patch[(kUH + 1) * (kUW + 1)];
-  __shared__ int row_a[kUH], row_b[kUH], col_a[kUW], col_b[kUW];
-  __shared__ float row_f[kUH], col_f[kUW];
-  const int64_t plane = blockIdx.z;
-  const int y0 = blockIdx.y * kTileH, x0 = blockIdx.x * kTileW;
+  const int64_t tid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (tid >= a.threads) return;
+  const int g = (int)(tid % a.groups);
+  const int64_t rest = tid / a.groups;
+  const int strip = (int)(rest % a.strips);
+  const int64_t plane = rest / a.strips;
+  const int x0 = 4 * g, y0 = strip * kRows;
   const float* __restrict__ lr = a.x_lr + plane * a.h * a.w;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int cx = 4 * tx;  // first tile column of this thread
-  const int x = x0 + cx;
-  // The noise this thread blends, requested first so that its DRAM latency
-  // overlaps the upsampling below.
-  float4 nz[4];
+  const int64_t obase = plane * a.H * (int64_t)a.W;
+
+  // noise of the strip, first
+  float4 nz[kRows];
   if (VEC) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int y = y0 + ty + 8 * k;
-      nz[k] = (y < a.H && x + 3 < a.W)
-                  ? __ldcs(reinterpret_cast<const float4*>(a.noise +
-                                                           (plane * a.H + y) * (int64_t)a.W + x))
+    for (int k = 0; k < kRows; ++k)
+      nz[k] = (y0 + k < a.H)
+                  ? __ldcs(reinterpret_cast<const float4*>(a.noise + obase +
+                                                           (int64_t)(y0 + k) * a.W + x0))
                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // Source coordinate of high-res index d along an axis of n low-res
+  // samples: (d + 0.5) / s - 0.5 = (2d + 1 - s) / (2s), integer part and
+  // fraction from the exact integer numerator.  Taps advance incrementally:
+  // from index d to d+1 the numerator grows by 2 and carries into the
+  // integer part at 2s, so only the first index of a run needs a division.
+  const int den = 2 * a.s;
+  const float inv_den = 1.0f / (float)den;
+  // column taps of x0-1 .. x0+4, clamped to the image
+  int ca[6], cb[6];
+  float cf[6];
+  {
+    const int xs = max(x0 - 1, 0);
+    int num = 2 * xs + 1 - a.s;
+    int fl = num >= 0 ? num / den : -((-num + den - 1) / den);
+    int rem = num - fl * den;
+    int x = xs;
+#pragma unroll
+    for (int j = 0; j < 6; ++j) {
+      if (x0 - 1 + j > x && x < a.W - 1) {  // advance to column x0-1+j (clamped)
+        ++x;
+        rem += 2;
+        if (rem >= den) {
+          rem -= den;
+          ++fl;
+        }
+      }
+      ca[j] = min(max(fl, 0), a.w - 1);
+      cb[j] = min(max(fl + 1, 0), a.w - 1);
+      cf[j] = (float)rem * inv_den;
     }
   }
-
-  // Source taps of the tile's rows and columns (with the halo, clamped to
-  // the image), once per CTA.
-  for (int i = threadIdx.x; i < kUH + kUW; i += kThreads) {
-    if (i < kUH) {
-      taps(min(max(y0 - 1 + i, 0), a.H - 1), a.s, a.h, row_a[i], row_b[i], row_f[i]);
-    } else {
-      const int c = i - kUH;
-      taps(min(max(x0 - 1 + c, 0), a.W - 1), a.s, a.w, col_a[c], col_b[c], col_f[c]);
+  // one low-res row interpolated at the 6 columns
+  auto hrow = [&](int r, float* hv) {
+    const float* row = lr + (int64_t)r * a.w;
+#pragma unroll
+    for (int j = 0; j < 6; ++j) hv[j] = __ldg(row + ca[j]) * (1.f - cf[j]) + __ldg(row + cb[j]) * cf[j];
+  };
+  int ra = -1, rb = -1;  // low-res rows held in ha, hb
+  float ha[6], hb[6];
+  // row taps, advanced one row per call from row max(y0-1, 0) (clamped
+  // at the last row)
+  int ry = max(y0 - 1, 0);
+  int rnum = 2 * ry + 1 - a.s;
+  int rfl = rnum >= 0 ? rnum / den : -((-rnum + den - 1) / den);
+  int rrem = rnum - rfl * den;
+  // u at high-res row y (clamped) and the 6 columns; y never decreases
+  auto urow = [&](int y, float* u) {
+    const int yc = min(max(y, 0), a.H - 1);
+    while (ry < yc) {
+      ++ry;
+      rrem += 2;
+      if (rrem >= den) {
+        rrem -= den;
+        ++rfl;
+      }
     }
-  }
-  __syncthreads();
-  // The low-res rectangle the taps reach, staged once with coalesced loads.
-  const int r0 = row_a[0], pr = row_b[kUH - 1] - r0 + 1;
-  const int c0 = col_a[0], pc = col_b[kUW - 1] - c0 + 1;
-  for (int i = threadIdx.x; i < pr * pc; i += kThreads) {
-    const int r = i / pc, c = i - (i / pc) * pc;
-    patch[i] = __ldg(lr + (int64_t)(r0 + r) * a.w + c0 + c);
-  }
-  __syncthreads();
-  // u on the tile and its halo.
-  for (int i = threadIdx.x; i < kUH * kUW; i += kThreads) {
-    const int r = i / kUW, c = i - (i / kUW) * kUW;
-    const float fy = row_f[r], fx = col_f[c];
-    const int xa = col_a[c] - c0, xb = col_b[c] - c0;
-    const float* ra = patch + (row_a[r] - r0) * pc;
-    const float* rb = patch + (row_b[r] - r0) * pc;
-    const float top = ra[xa] * (1.f - fx) + ra[xb] * fx;
-    const float bot = rb[xa] * (1.f - fx) + rb[xb] * fx;
-    u[r][c] = top * (1.f - fy) + bot * fy;
-  }
-  __syncthreads();
-
+    const int ya = min(max(rfl, 0), a.h - 1), yb = min(max(rfl + 1, 0), a.h - 1);
+    const float fy = (float)rrem * inv_den;
+    if (ya != ra) {
+      if (ya == rb) {
+#pragma unroll
+        for (int j = 0; j < 6; ++j) ha[j] = hb[j];
+      } else {
+        hrow(ya, ha);
+      }
+      ra = ya;
+    }
+    if (yb != rb) {
+      hrow(yb, hb);
+      rb = yb;
+    }
+#pragma unroll
+    for (int j = 0; j < 6; ++j) u[j] = ha[j] * (1.f - fy) + hb[j] * fy;
+  };
+  // horizontal blur of u at the 4 output columns
+  auto hblur = [](const float* u, float* b) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b[j] = 0.25f * u[j] + 0.5f * u[j + 1] + 0.25f * u[j + 2];
+  };
+  float u_cur[6], u_nxt[6], b_prev[4], b_cur[4], b_nxt[4];
+  urow(y0 - 1, u_cur);
+  hblur(u_cur, b_prev);
+  urow(y0, u_cur);
+  hblur(u_cur, b_cur);
   const float keep = 1.f + a.amount, t1 = 1.f - a.t;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int ry = ty + 8 * k;  // tile row
-    const int y = y0 + ry;
+  for (int k = 0; k < kRows; ++k) {
+    const int y = y0 + k;
     if (y >= a.H) break;
-    float hb[3][4];  // horizontal blur of the three rows around ry
-#pragma unroll
-    for (int dy = 0; dy < 3; ++dy) {
-      const float* row = &u[ry + dy][cx];
-      float v[6];
-#pragma unroll
-      for (int j = 0; j < 6; ++j) v[j] = row[j];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) hb[dy][j] = 0.25f * v[j] + 0.5f * v[j + 1] + 0.25f * v[j + 2];
-    }
+    urow(y + 1, u_nxt);
+    hblur(u_nxt, b_nxt);
     float res[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float b = 0.25f * hb[0][j] + 0.5f * hb[1][j] + 0.25f * hb[2][j];
-      const float c = u[ry + 1][cx + 1 + j];
-      res[j] = t1 * (keep * c - a.amount * b);
+      const float bl = 0.25f * b_prev[j] + 0.5f * b_cur[j] + 0.25f * b_nxt[j];
+      res[j] = t1 * (keep * u_cur[j + 1] - a.amount * bl);
     }
-    const int64_t off = (plane * a.H + y) * (int64_t)a.W + x;
-    if (VEC && x + 3 < a.W) {
-      const float4 n = nz[k];
-      float4 o;
-      o.x = fmaf(a.t, n.x, res[0]);
-      o.y = fmaf(a.t, n.y, res[1]);
-      o.z = fmaf(a.t, n.z, res[2]);
-      o.w = fmaf(a.t, n.w, res[3]);
-      __stcs(reinterpret_cast<float4*>(a.out + off), o);
+    const int64_t off = obase + (int64_t)y * a.W + x0;
+    if (VEC) {
+      if (x0 + 3 < a.W) {
+        float4 o;
+        o.x = fmaf(a.t, nz[k].x, res[0]);
+        o.y = fmaf(a.t, nz[k].y, res[1]);
+        o.z = fmaf(a.t, nz[k].z, res[2]);
+        o.w = fmaf(a.t, nz[k].w, res[3]);
+        __stcs(reinterpret_cast<float4*>(a.out + off), o);
+      }
     } else {
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        if (x + j < a.W) a.out[off + j] = fmaf(a.t, __ldcs(a.noise + off + j), res[j]);
+        if (x0 + j < a.W) a.out[off + j] = fmaf(a.t, __ldcs(a.noise + off + j), res[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 6; ++j) u_cur[j] = u_nxt[j];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      b_prev[j] = b_cur[j];
+      b_cur[j] = b_nxt[j];
     }
   }
 }
@@ -165,12 +199,14 @@ int launch_warm_start(const ug_warm_start_params* p, const float* x_lr, const fl
   a.W = p->lr_w * p->scale;
   a.amount = p->sharpen;
   a.t = p->t;
-  const dim3 grid((a.W + kTileW - 1) / kTileW, (a.H + kTileH - 1) / kTileH,
-                  (unsigned)(p->batch * p->channels));
+  a.groups = (a.W + 3) / 4;
+  a.strips = (a.H + kRows - 1) / kRows;
+  a.threads = (int64_t)p->batch * p->channels * a.strips * a.groups;
+  const int64_t blocks = (a.threads + kThreads - 1) / kThreads;
   if (a.W % 4 == 0)
-    warm_start_kernel<true><<<grid, kThreads, 0, st>>>(a);
+    warm_start_kernel<true><<<(unsigned)blocks, kThreads, 0, st>>>(a);
   else
-    warm_start_kernel<false><<<grid, kThreads, 0, st>>>(a);
+    warm_start_kernel<false><<<(unsigned)blocks, kThreads, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? UG_OK : UG_ERR_CUDA;
 }
 
