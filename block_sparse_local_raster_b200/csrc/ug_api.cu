@@ -70,6 +70,70 @@ int ug_visible_pairs(const ug_geom* g, int64_t* hr_hr, int64_t* hr_lr, int64_t* 
   return UG_OK;
 }
 
+namespace {
+
+int work_lists(const ug_geom* g, std::vector<QTile>& qt, std::vector<uint32_t>& kv,
+               std::vector<KTile>& kt, std::vector<uint32_t>& ql) {
+  int st = validate(g);
+  if (st != UG_OK) return st;
+  std::vector<int32_t> off, idx;
+  build_neighbours(*g, off, idx);
+  int32_t nhr, nlr;
+  build_attention_lists(*g, off, idx, qt, kv, &nhr, &nlr);
+  build_backward_lists(*g, off, idx, kt, ql);
+  return UG_OK;
+}
+
+}  // namespace
+
+int ug_work_list_sizes(const ug_geom* g, int64_t* n_qctas, int64_t* n_kvlist, int64_t* n_kctas,
+                       int64_t* n_qlist) {
+  std::vector<QTile> qt;
+  std::vector<uint32_t> kv, ql;
+  std::vector<KTile> kt;
+  int st;
+  try {
+    st = work_lists(g, qt, kv, kt, ql);
+  } catch (...) {
+    return UG_ERR_NO_MEMORY;
+  }
+  if (st != UG_OK) return st;
+  if (n_qctas) *n_qctas = (int64_t)qt.size();
+  if (n_kvlist) *n_kvlist = (int64_t)kv.size();
+  if (n_kctas) *n_kctas = (int64_t)kt.size();
+  if (n_qlist) *n_qlist = (int64_t)ql.size();
+  return UG_OK;
+}
+
+int ug_build_work_lists(const ug_geom* g, int32_t* qctas, uint32_t* kvlist, int32_t* kctas,
+                        uint32_t* qlist) {
+  std::vector<QTile> qt;
+  std::vector<uint32_t> kv, ql;
+  std::vector<KTile> kt;
+  int st;
+  try {
+    st = work_lists(g, qt, kv, kt, ql);
+  } catch (...) {
+    return UG_ERR_NO_MEMORY;
+  }
+  if (st != UG_OK) return st;
+  for (size_t i = 0; qctas && i < qt.size(); ++i) {
+    qctas[4 * i] = qt[i].lowres;
+    qctas[4 * i + 1] = qt[i].q0;
+    qctas[4 * i + 2] = qt[i].list_off;
+    qctas[4 * i + 3] = qt[i].list_len;
+  }
+  for (size_t i = 0; kctas && i < kt.size(); ++i) {
+    kctas[4 * i] = kt[i].lowres;
+    kctas[4 * i + 1] = kt[i].k0;
+    kctas[4 * i + 2] = kt[i].list_off;
+    kctas[4 * i + 3] = kt[i].list_len;
+  }
+  if (kvlist) std::memcpy(kvlist, kv.data(), kv.size() * sizeof(uint32_t));
+  if (qlist) std::memcpy(qlist, ql.data(), ql.size() * sizeof(uint32_t));
+  return UG_OK;
+}
+
 const char* ug_status_string(int s) {
   switch (s) {
     case UG_OK: return "ok";

@@ -33,6 +33,7 @@ UG_LR = 2
 # Every symbol include/ug.h declares.
 EXPORTS = (
     "ug_geom_validate", "ug_index_map_sizes", "ug_build_index_maps", "ug_visible_pairs",
+    "ug_work_list_sizes", "ug_build_work_lists",
     "ug_status_string", "ug_plan_create", "ug_plan_destroy", "ug_get_index_maps",
     "ug_permute_window_first", "ug_permute_rope_window_first", "ug_unpermute", "ug_rope_2d",
     "ug_hier_local_attn_fwd", "ug_hier_local_attn_fwd_vo_raster",
@@ -93,6 +94,9 @@ def lib() -> ctypes.CDLL:
         "ug_index_map_sizes": (I32, [G, pi64, pi64, pi64]),
         "ug_build_index_maps": (I32, [G, pi32, pi32, pi32]),
         "ug_visible_pairs": (I32, [G, pi64, pi64, pi64]),
+        "ug_work_list_sizes": (I32, [G, pi64, pi64, pi64, pi64]),
+        "ug_build_work_lists": (I32, [G, pi32, ctypes.POINTER(ctypes.c_uint32), pi32,
+                                      ctypes.POINTER(ctypes.c_uint32)]),
         "ug_status_string": (ctypes.c_char_p, [I32]),
         "ug_plan_create": (I32, [G, ctypes.POINTER(P)]),
         "ug_plan_destroy": (I32, [P]),
@@ -153,6 +157,22 @@ def build_index_maps(g: ug_geom):
     ptrs = [a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) for a in arrs]
     _check(lib().ug_build_index_maps(ctypes.byref(g), *ptrs), "ug_build_index_maps")
     return tuple(arrs)
+
+
+def work_lists(g: ug_geom):
+    """(qctas [n, 4], kvlist, kctas [m, 4], qlist) as numpy arrays (host only)."""
+    n = [ctypes.c_int64() for _ in range(4)]
+    _check(lib().ug_work_list_sizes(ctypes.byref(g), *[ctypes.byref(x) for x in n]),
+           "ug_work_list_sizes")
+    qc = np.zeros((n[0].value, 4), dtype=np.int32)
+    kv = np.zeros(n[1].value, dtype=np.uint32)
+    kc = np.zeros((n[2].value, 4), dtype=np.int32)
+    ql = np.zeros(n[3].value, dtype=np.uint32)
+    p32 = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    pu32 = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint32))
+    _check(lib().ug_build_work_lists(ctypes.byref(g), p32(qc), pu32(kv), p32(kc), pu32(ql)),
+           "ug_build_work_lists")
+    return qc, kv, kc, ql
 
 
 def visible_pairs(g: ug_geom):

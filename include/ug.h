@@ -120,6 +120,28 @@ int ug_build_index_maps(const ug_geom* g, int32_t* perm, int32_t* nbr_off, int32
  * useful FLOPs of the attention are 4 * head_dim * heads * batch * (sum). */
 int ug_visible_pairs(const ug_geom* g, int64_t* hr_hr, int64_t* hr_lr, int64_t* lr_lr);
 
+/* Element counts of the attention work lists of ug_build_work_lists. */
+int ug_work_list_sizes(const ug_geom* g, int64_t* n_qctas, int64_t* n_kvlist, int64_t* n_kctas,
+                       int64_t* n_qlist);
+
+/* The work lists the attention kernels walk, into caller-owned host arrays
+ * (sizes from ug_work_list_sizes; any pointer may be NULL):
+ *   qctas  (4 per forward query CTA): token set (0 high-res, 1 global), first
+ *          query row, offset and length of its slice of kvlist.  A CTA owns
+ *          256 rows (two 128-row tiles) of its token set.
+ *   kvlist: one entry per 128-key block a CTA must visit: bits 0-28 the block
+ *          index (keys [128 i, 128 i + 128) of its tensor), bit 29 set for
+ *          the global tensor, bit 30 set when some in-range (query, key) pair
+ *          of the CTA and block is invisible or a block or CTA passes the end
+ *          of its tensor (the kernel then tests each pair).
+ *   kctas  (4 per backward key CTA): token set, first key, offset and length
+ *          of its slice of qlist.
+ *   qlist: one entry per 128-row query tile a key CTA must visit, same bit
+ *          layout; bit 30 marks an invisible in-range pair.
+ * Host only, no GPU needed. */
+int ug_build_work_lists(const ug_geom* g, int32_t* qctas, uint32_t* kvlist, int32_t* kctas,
+                        uint32_t* qlist);
+
 const char* ug_status_string(int status);
 
 /* ---- plan ---------------------------------------------------------------- */
