@@ -76,8 +76,13 @@ def test_attention_backward_every_element(name):
         check(got, r, b, f"{name} {what}")
 
 
-def test_attention_backward_sampled_4k():
-    wl = workloads.get("4K")
+@pytest.mark.parametrize("name", ["4K", "4K-CFG", "4K-text"])
+def test_attention_backward_sampled_full_size(name):
+    """Full-size layers: sampled query rows (dQ) and high-res keys (dK, dV)
+    of two heads against the oracle under the derived bounds, plus the
+    gradient-sum identities for every head and key.  4K-CFG adds batch 2
+    and per-head scales of q, k, v; 4K-text adds 512 text tokens."""
+    wl = workloads.get(name)
     g = ogeom(wl)
     p = plan(wl)
     x = inputs(wl, 810)
@@ -86,7 +91,13 @@ def test_attention_backward_sampled_4k():
     rows = np.concatenate([sample_hr_tokens(g, O.HR_WINDOW_FIRST, 5, n_interior=2, per_window=2),
                            g.N + sample_lr_tokens(g, 5, n=4)])
     T, nx = g.T, g.n_win_x
-    keys = np.array([0, T - 1, (7 * nx + 9) * T + 100, g.N - 1])  # corner, interior, last window
+    mid = (g.n_win_y // 2) * nx + nx // 2
+    # corner, interior and last window at 4K, the corner key with text
+    # tokens; a key's dK, dV need the full rows of every query that sees it,
+    # so the 1024-token windows of 4K-CFG (17k such rows) check dQ rows and
+    # the identities only
+    keys = (np.array([0, mid * T + min(100, T - 1), g.N - 1]) if name == "4K"
+            else np.array([0]) if T <= 256 else np.zeros(0, dtype=np.int64))
     xb = {k: bits(v[:, :, heads]) for k, v in x.items()}
     g1 = O.Geometry.from_dict(dict(wl.geom_dict(), heads=len(heads)))
     ref = O.attention_backward(xb["q_hr"], xb["k_hr"], xb["v_hr"], xb["q_lr"], xb["k_lr"],
@@ -96,9 +107,10 @@ def test_attention_backward_sampled_4k():
                            *(joint_f64(x, n, heads) for n in ("q", "k", "v", "do")),
                            rows=rows, keys=keys)
     gq, gk, gv = joint_grads(grads, wl, heads)
-    check(gq[:, rows], ref[0], bnd[0], "4K dq")
-    check(gk[:, keys], ref[1], bnd[1], "4K dk")
-    check(gv[:, keys], ref[2], bnd[2], "4K dv")
+    check(gq[:, rows], ref[0], bnd[0], f"{name} dq")
+    if keys.size:
+        check(gk[:, keys], ref[1], bnd[1], f"{name} dk")
+        check(gv[:, keys], ref[2], bnd[2], f"{name} dv")
     # identities of any softmax attention, all heads, every key (sums in fp64
     # on the device)
     tot = lambda a, b_: a.double().sum(1) + b_.double().sum(1)
