@@ -372,23 +372,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // p = 2^(s*scale*log2e - m): fp32 row sum; bf16 pairs (even key in the
-      // low half) over the first 64 columns of S_t, the A operand of O += P V.
+      // low half) over the first 64 columns of S_t, the A operand of O += P V,
+      // stored 8 columns at a time so that few packed values are live next to
+      // the 128 scores (no register spills).
       const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
       const float2 nm2 = make_float2(-m_use, -m_use);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
+      for (int h = 0; h < 8; ++h) {
+        uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          const int k = 64 * h + i;
+        for (int i = 0; i < 16; i += 2) {
+          const int k = 16 * h + i;
           const float2 x = __ffma2_rn(make_float2(s[k], s[k + 1]), sc2, nm2);
           const float2 pp = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-          acc[(i / 2) & 3] = __fadd2_rn(acc[(i / 2) & 3], pp);
+          acc[(k / 2) & 3] = __fadd2_rn(acc[(k / 2) & 3], pp);
           pk[i / 2] = pack_bf16(pp.x, pp.y);
         }
-        tmem_st32u(tS + 32 * h, pk);
+        tmem_st8u(tS + 8 * h, pk);
       }
       const float2 a4 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
       l = l * alpha + (a4.x + a4.y);
