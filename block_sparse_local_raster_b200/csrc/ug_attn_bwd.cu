@@ -12,8 +12,9 @@
 //   dq_kernel     one 128-row query tile per CTA; Q and dO stay in shared
 //                 memory while K_j, V_j stream through a 5-slot TMA ring over
 //                 the forward's key-block list; per block S = Q K^T and
-//                 dP = dO V^T share one TMEM buffer, and dS (bf16, written
-//                 over it) is the TMEM A operand of dQ += dS K;
+//                 dP = dO V^T share one TMEM buffer, P (bf16) waits for dP in
+//                 the TMEM quarter the layout leaves free, and dS (bf16,
+//                 written over S/dP) is the TMEM A operand of dQ += dS K;
 //   dkv_kernel    one 128-key block per CTA; K and V stay in shared memory
 //                 while Q_i, dO_i stream over the block's list of query
 //                 tiles; S^T = K Q_i^T gives P^T (bf16 in TMEM), the A
