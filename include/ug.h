@@ -50,7 +50,7 @@ extern "C" {
 typedef enum ug_status {
   UG_OK = 0,
   UG_ERR_INVALID_ARG = 1,  /* null pointer, bad geometry, bad token set         */
-  UG_ERR_UNSUPPORTED = 2,  /* a valid geometry this build does not run          */
+  UG_ERR_UNSUPPORTED = 2,  /* a valid geometry the library does not run        */
   UG_ERR_ALIGNMENT = 3,    /* a device pointer not 16-byte aligned              */
   UG_ERR_ALIAS = 4,        /* output overlaps an input where that is not allowed */
   UG_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed                 */
