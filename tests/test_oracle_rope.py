@@ -132,3 +132,31 @@ def test_frequency_ladder():
     want = np.array([10000.0 ** (-k / 8.0) for k in range(8)])  # a = 16 -> 2k/16 = k/8
     np.testing.assert_allclose(ang, want, rtol=1e-6)
     np.testing.assert_array_equal(tab["hr_y"][0][0], np.ones(8, np.float32))
+
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None)
+@given(st.sampled_from([16, 32, 64]), st.integers(0, 200), st.integers(0, 200),
+       st.integers(0, 200), st.integers(0, 999))
+def test_random_positions_rotation_properties(a, p1, p2, shift, seed):
+    """One axis of a positions p1, p2 (exact fp64 rotation before rounding):
+    pair norms are preserved, <R(p1) x, R(p2) y> depends only on p2 - p1
+    up to the fp32 rounding of cos and sin, and the transpose is the adjoint."""
+    rng = np.random.default_rng(seed)
+    f = O.rope_frequencies(a, 10000.0)
+    c, s_ = O._cos_sin_table([float(p1), float(p2), float(p1 + shift), float(p2 + shift)], f)
+    c, s_ = c.astype(np.float64), s_.astype(np.float64)
+    x = rng.standard_normal(a)
+    y = rng.standard_normal(a)
+    rx = O.rope_rotate_f64(x, c[0], s_[0])
+    np.testing.assert_allclose(np.hypot(rx[0::2], rx[1::2]), np.hypot(x[0::2], x[1::2]),
+                               rtol=1e-6)
+    ry = O.rope_rotate_f64(y, c[1], s_[1])
+    rx2 = O.rope_rotate_f64(x, c[2], s_[2])
+    ry2 = O.rope_rotate_f64(y, c[3], s_[3])
+    np.testing.assert_allclose(rx @ ry, rx2 @ ry2, rtol=0, atol=1e-5 * (1 + abs(rx @ ry)))
+    np.testing.assert_allclose(rx @ y, x @ O.rope_rotate_f64(y, c[0], -s_[0]), rtol=0,
+                               atol=1e-12)

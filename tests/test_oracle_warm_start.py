@@ -74,3 +74,21 @@ def test_two_by_two_worked_by_hand():
     want = row[:, None] + col[None, :]
     out = W.warm_start(x, np.zeros((1, 1, 4, 4)), 2, 1.0, 0.0)[0, 0]
     np.testing.assert_array_equal(out, want)
+
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None)
+@given(st.integers(1, 9), st.integers(1, 9), st.integers(1, 6), st.integers(0, 999))
+def test_random_shapes_reduce_to_torch_bilinear(h, w, s, seed):
+    """With no sharpening and t = 0 the state is the bilinear upsample, for
+    any size and integer factor; with t = 1 it is the noise."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((1, 2, h, w))
+    noise = rng.standard_normal((1, 2, h * s, w * s))
+    want = F.interpolate(torch.from_numpy(x), scale_factor=s, mode="bilinear",
+                         align_corners=False).numpy()
+    np.testing.assert_allclose(W.warm_start(x, noise, s, 0.0, 0.0), want, rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(W.warm_start(x, noise, s, 0.7, 1.0), noise)
