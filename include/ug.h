@@ -132,8 +132,9 @@ int ug_work_list_sizes(const ug_geom* g, int64_t* n_qctas, int64_t* n_kvlist, in
  *   kvlist: one entry per 128-key block a CTA must visit: bits 0-28 the block
  *          index (keys [128 i, 128 i + 128) of its tensor), bit 29 set for
  *          the global tensor, bit 30 set when some in-range (query, key) pair
- *          of the CTA and block is invisible or a block or CTA passes the end
- *          of its tensor (the kernel then tests each pair).
+ *          of the CTA and block is invisible or the block passes the end of
+ *          its tensor (the kernel then tests each pair; rows past the end of
+ *          the query tensor are computed but never written).
  *   kctas  (4 per backward key CTA): token set, first key, offset and length
  *          of its slice of qlist.
  *   qlist: one entry per 128-row query tile a key CTA must visit, same bit
