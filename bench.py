@@ -12,9 +12,13 @@ metric is useful attention TFLOP/s
 ms per layer; the attention kernel alone is also timed and set against the
 measured bf16 tensor peak.
 
+The default run times the 4K layer (the JSON line's value), then in the same
+process the 2K, 8K and 4K-CFG layers (``per_config``) and the 4K layer's
+backward pass (``backward``), each with its own clock record and roofline.
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4K] [--impl ug|reference]
   python bench.py --op warm_start [--config 4K|8K]   (the warm-start kernel alone)
-  python bench.py --op backward [--config 4K]        (the layer's backward pass)
+  python bench.py --op backward [--config 4K]        (the layer's backward pass alone)
 
 N > 1 runs under torchrun, one rank per GPU; every rank runs its own layer on
 its own inputs (independent problems, weak scaling, no data-path collective);
@@ -57,6 +61,10 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=12)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default="layer", choices=["layer", "warm_start", "backward"])
+    ap.add_argument("--per-config", default="2K,8K,4K-CFG",
+                    help="configs timed after the main one in the same run ('' = none)")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward pass timed after the main layer")
     return ap.parse_args()
 
 
@@ -108,53 +116,140 @@ def aggregate(units_per_rank: float, world: int, max_seconds: float) -> float:
     return units_per_rank * world / max_seconds
 
 
+def _nvml_handle(device_index: int):
+    """NVML handle of the CUDA device (by UUID, else PCI bus id)."""
+    import pynvml
+    pynvml.nvmlInit()
+    props = torch.cuda.get_device_properties(device_index)
+    tries = []
+    u = str(getattr(props, "uuid", ""))
+    if u:
+        tries += [lambda: pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)]
+    if hasattr(props, "pci_bus_id"):
+        bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+        tries += [lambda: pynvml.nvmlDeviceGetHandleByPciBusId(bus)]
+    for t in tries:
+        try:
+            return t()
+        except Exception:
+            continue
+    raise RuntimeError("no NVML handle for this device")
+
+
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clock, power and clock-event reasons sampled during the timed
+    region, read-only: NVML every 10 ms from a thread (nvidia-smi at 20 ms if
+    NVML is unavailable)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    SMI = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+           "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+           "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.dev = device_index
+        self.period = period_s
+        self.rows = []  # (sm_mhz, sm_max_mhz, power_w, reason bits)
+        self.thread = None
         self.proc = None
-        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.stop_flag = False
+        self.source = None
+
+    def _nvml_loop(self, h):
+        import pynvml
+        smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stop_flag:
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append((float(sm), float(smax), pw, int(rs)))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
         try:
+            import threading
+            h = _nvml_handle(self.dev)
+            self.thread = threading.Thread(target=self._nvml_loop, args=(h,), daemon=True)
+            self.thread.start()
+            self.source = "nvml, 10 ms"
+            return
+        except Exception:
+            self.thread = None
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.SMI}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=self.out, stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, 20 ms"
         except OSError:
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.out.flush()
-        rows = [l.split(", ") for l in open(self.out.name).read().strip().splitlines() if l]
-        os.unlink(self.out.name)
-        sm, smax, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+        elif self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(r[1]))
-                smax = max(smax, float(r[2]))
-                for n, v in zip(names, r[5:9]):
-                    if v.strip() == "Active":
-                        reasons.add(n)
-            except (ValueError, IndexError):
-                continue
-        if not sm:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.flush()
+            for line in open(self.out.name).read().strip().splitlines():
+                r = line.split(", ")
+                try:
+                    bits = sum(b for (_, b), v in zip(self.REASONS, r[5:9]) if v.strip() == "Active")
+                    self.rows.append((float(r[1]), float(r[2]), float(r[3]), bits))
+                except (ValueError, IndexError):
+                    continue
+            os.unlink(self.out.name)
+        else:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return self.summary(self.rows)
+
+    def summary(self, rows):
+        if not rows:
+            return None
+        sm = [r[0] for r in rows]
+        reasons = sorted({n for r in rows for n, b in self.REASONS if r[3] & b})
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": round(max(r[2] for r in rows), 1),
+                "reasons": reasons, "samples": len(rows), "source": self.source}
+
+
+def pick_peak(pk, region_s: float, clk):
+    """The bf16 peak that applies to a kernel timed over region_s seconds.
+
+    The burst figure (cuBLAS timed alone, full clock) unless the region is a
+    second or longer and its clock record shows the power cap or a median SM
+    clock below 95 % of max: then the sustained figure (cuBLAS after seconds
+    under the power cap).  Returns (peak, kind)."""
+    throttled = clk is not None and ("sw_power_cap" in clk["reasons"]
+                                     or clk["sm_mhz"] < 0.95 * clk["sm_max_mhz"])
+    if region_s >= 1.0 and throttled:
+        return pk["bf16_tflops_sustained"], "sustained"
+    return pk["bf16_tflops"], "burst"
+
+
+def tensor_roofline(achieved: float, region_s: float, clk, traffic=None, note=None):
+    pk, src = peaks()
+    peak, kind = pick_peak(pk, region_s, clk)
+    r = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+         "frac": achieved / peak, "traffic": traffic,
+         "peak_source": f"{src} bf16 cuBLAS, {kind} (timed region {region_s:.2f} s; "
+                        "burst below 1 s or at full clock without the power cap)",
+         "peak_kind": kind,
+         "frac_of_burst_peak": achieved / pk["bf16_tflops"],
+         "frac_of_sustained_peak": achieved / pk["bf16_tflops_sustained"]}
+    if note:
+        r["note"] = note
+    return r
 
 
 def attn_source_hash() -> str:
@@ -183,12 +278,21 @@ def attn_traffic_bytes(config: str):
 # ----------------------------------------------------------------------------- CPU oracle
 
 def cpu_threads() -> int:
+    """Threads the oracle's BLAS uses."""
     try:
         from threadpoolctl import threadpool_info
         n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
         return int(max(n)) if n else 1
     except Exception:
         return 1
+
+
+def cpu_cores() -> int:
+    """Host cores this process may run on (nproc)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 class OracleArm:
@@ -243,7 +347,7 @@ def run_reference(args, wl, world, rank):
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "sample": sample},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "nproc": cpu_cores(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -253,6 +357,147 @@ def run_reference(args, wl, world, rank):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+def _chk(st, what):
+    from block_sparse_local_raster_b200 import ug
+    if st != ug.UG_OK:
+        raise ug.UgError(st, what)
+
+
+class LayerRunner:
+    """One layer step on device-resident raster inputs `d`, launched as
+    ug_layer_fwd does but call by call, so that the attention launch can be
+    bracketed by its own CUDA events."""
+
+    def __init__(self, wl, d, dev, stream):
+        from block_sparse_local_raster_b200 import ug
+        self.ug, self.wl, self.d, self.stream = ug, wl, d, stream
+        self.plan = ug.Plan(**wl.geom_dict())
+        B, N, H, D = d["q_hr"].shape
+        L = self.L = wl.n_lr
+        self.ws = torch.empty(self.plan.workspace_bytes(), dtype=torch.uint8, device=dev)
+        self.o_hr = torch.empty_like(d["q_hr"])
+        self.o_lr = torch.empty_like(d["q_lr"]) if L else None
+        self.lse = torch.empty((B, H, N + L), dtype=torch.float32, device=dev)
+        self.hr_bytes = hb = d["q_hr"].numel() * 2
+        lb = d["q_lr"].numel() * 2
+        up = lambda n: (n + 255) // 256 * 256
+        ws = self.ws
+        view = lambda off, nb, n: ws[off:off + nb].view(torch.bfloat16).view(B, n, H, D)
+        # window-first scratch inside the workspace, same split as ug_layer_fwd
+        self.q_wf, self.k_wf = view(0, hb, N), view(up(hb), hb, N)
+        self.v_wf, self.o_wf = view(2 * up(hb), hb, N), view(3 * up(hb), hb, N)
+        o4 = 4 * up(hb)
+        self.ql = view(o4, lb, L) if L else None
+        self.kl = view(o4 + up(lb), lb, L) if L else None
+        # where 128-key tiles are whole window rows the attention reads v and
+        # writes o in raster order (no permute of v, no unpermute of o)
+        T = wl.win_h * wl.win_w
+        self.vo_raster = 128 % wl.win_w == 0 and T % 128 == 0
+        self.launches = 2 + (2 if L else 0) + 1 + (0 if self.vo_raster else 2)
+        self.flops = useful_flops(wl)
+
+    @staticmethod
+    def launches_of(wl) -> int:
+        T = wl.win_h * wl.win_w
+        vo = 128 % wl.win_w == 0 and T % 128 == 0
+        return 2 + (2 if wl.n_lr else 0) + 1 + (0 if vo else 2)
+
+    def step(self, ev=None):
+        ug, d, p, L = self.ug, self.d, self.plan, self.L
+        _chk(p.permute_rope_window_first(d["q_hr"], self.q_wf), "permute+rope q")
+        _chk(p.permute_rope_window_first(d["k_hr"], self.k_wf), "permute+rope k")
+        if not self.vo_raster:
+            _chk(p.permute_window_first(d["v_hr"], self.v_wf), "permute v")
+        if L:
+            _chk(p.rope_2d(d["q_lr"], self.ql, ug.UG_LR), "rope q_lr")
+            _chk(p.rope_2d(d["k_lr"], self.kl, ug.UG_LR), "rope k_lr")
+        if ev is not None:
+            ev[0].record(self.stream)
+        vl = d["v_lr"] if L else None
+        if self.vo_raster:
+            _chk(p.hier_local_attn_fwd_vo_raster(self.q_wf, self.k_wf, d["v_hr"], self.ql,
+                                                 self.kl, vl, self.o_hr, self.o_lr, self.lse),
+                 "attention")
+        else:
+            _chk(p.hier_local_attn_fwd(self.q_wf, self.k_wf, self.v_wf, self.ql, self.kl, vl,
+                                       self.o_wf, self.o_lr, self.lse), "attention")
+        if ev is not None:
+            ev[1].record(self.stream)
+        if not self.vo_raster:
+            _chk(p.unpermute(self.o_wf, self.o_hr), "unpermute")
+
+    def close(self):
+        self.plan.close()
+
+
+def time_steps(step, steps, warmup, dev, stream, rank, local, per_step_flush_bytes=0):
+    """W untimed steps, then exactly `steps` timed ones between a barrier and
+    a device synchronise on both sides, with the clocks sampled meanwhile.
+    step(ev) records ev[0] / ev[1] around the kernel it wants timed alone.
+    When the inputs fit in L2 (per_step_flush_bytes > 0) a buffer of that
+    size is written between steps and each step is timed by its own events,
+    so the flush is outside the time.  Returns (seconds per step, kernel
+    seconds per launch, clock record), max over ranks."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    flush = (torch.empty(per_step_flush_bytes, dtype=torch.uint8, device=dev)
+             if per_step_flush_bytes else None)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    kev = [(mk(), mk()) for _ in range(steps)]
+    sev = [(mk(), mk()) for _ in range(steps)] if flush is not None else None
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.05)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = mk(), mk()
+    t0.record(stream)
+    for i in range(steps):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+            sev[i][0].record(stream)
+        step(kev[i])
+        if flush is not None:
+            sev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    if sev is not None:
+        sec = sum(a.elapsed_time(b) for a, b in sev) / 1e3 / steps
+    else:
+        sec = t0.elapsed_time(t1) / 1e3 / steps
+    ksec = sum(a.elapsed_time(b) for a, b in kev) / 1e3 / steps
+    return reduce_max(sec, dev), reduce_max(ksec, dev), clk
+
+
+def layer_record(args, wl, d, dev, stream, rank, local, steps=None, warmup=None):
+    """Times the layer on device inputs d; returns (runner, record dict)."""
+    r = LayerRunner(wl, d, dev, stream)
+    steps = steps or args.steps
+    warmup = warmup if warmup is not None else args.warmup
+    flush = 0 if r.hr_bytes > L2_BYTES else 2 * L2_BYTES
+    sec, attn, clk = time_steps(r.step, steps, warmup, dev, stream, rank, local, flush)
+    _chk(r.plan.check_error(), f"{wl.name} timed steps")
+    ach = r.flops / attn / 1e12
+    rec = {
+        "ms_per_layer": sec * 1e3, "layer_tflops": r.flops / sec / 1e12,
+        "attn_ms": attn * 1e3, "attn_tflops": ach, "steps": steps, "warmup": warmup,
+        "useful_flop_per_layer": r.flops,
+        "l2": ("inputs larger than L2 (each high-res tensor %.0f MB > 126 MB), no flush"
+               % (r.hr_bytes / 1e6)) if not flush else
+              ("inputs smaller than L2 (%.0f MB per high-res tensor): a %d MB buffer is "
+               "written between steps, outside each step's events" % (r.hr_bytes / 1e6,
+                                                                       flush >> 20)),
+        "roofline": tensor_roofline(ach, attn * steps, clk,
+                                    attn_traffic_bytes(wl.name)),
+        "clocks": clk,
+    }
+    return r, rec
+
+
 def run_ug(args, wl, world, rank, local):
     from block_sparse_local_raster_b200 import ug
     torch.cuda.set_device(local)
@@ -260,94 +505,16 @@ def run_ug(args, wl, world, rank, local):
     init_dist("nccl", world)
     stream = torch.cuda.current_stream(dev)
 
-    plan = ug.Plan(**wl.geom_dict())
     host = workloads.make_inputs(wl, seed=rank)
     host.pop("head_scale", None)
     pinned = {k: v.pin_memory() for k, v in host.items()}
     d = {k: v.to(dev) for k, v in pinned.items()}
-    B, N, H, D = d["q_hr"].shape
     L = wl.n_lr
-    ws = torch.empty(plan.workspace_bytes(), dtype=torch.uint8, device=dev)
-    o_hr = torch.empty_like(d["q_hr"])
-    o_lr = torch.empty_like(d["q_lr"]) if L else None
-    lse = torch.empty((B, H, N + L), dtype=torch.float32, device=dev)
-    hr_bytes = d["q_hr"].numel() * 2
-    lr_bytes = d["q_lr"].numel() * 2
-    up = lambda n: (n + 255) // 256 * 256
-    # window-first scratch inside the workspace, same split as ug_layer_fwd
-    ws_q = ws[0:hr_bytes].view(torch.bfloat16).view(B, N, H, D)
-    ws_k = ws[up(hr_bytes):up(hr_bytes) + hr_bytes].view(torch.bfloat16).view(B, N, H, D)
-    ws_v = ws[2 * up(hr_bytes):2 * up(hr_bytes) + hr_bytes].view(torch.bfloat16).view(B, N, H, D)
-    ws_o = ws[3 * up(hr_bytes):3 * up(hr_bytes) + hr_bytes].view(torch.bfloat16).view(B, N, H, D)
-    o4 = 4 * up(hr_bytes)
-    ws_ql = ws[o4:o4 + lr_bytes].view(torch.bfloat16).view(B, L, H, D) if L else None
-    ws_kl = ws[o4 + up(lr_bytes):o4 + up(lr_bytes) + lr_bytes].view(torch.bfloat16).view(B, L, H, D) if L else None
-
-    def chk(st, what):
-        if st != ug.UG_OK:
-            raise ug.UgError(st, what)
-
-    # where 128-key tiles are whole window rows the attention reads v and
-    # writes o in raster order (no permute of v, no unpermute of o)
-    T = wl.win_h * wl.win_w
-    vo_raster = 128 % wl.win_w == 0 and T % 128 == 0
-
-    def step(ev=None):
-        chk(plan.permute_rope_window_first(d["q_hr"], ws_q), "permute+rope q")
-        chk(plan.permute_rope_window_first(d["k_hr"], ws_k), "permute+rope k")
-        if not vo_raster:
-            chk(plan.permute_window_first(d["v_hr"], ws_v), "permute v")
-        if L:
-            chk(plan.rope_2d(d["q_lr"], ws_ql, ug.UG_LR), "rope q_lr")
-            chk(plan.rope_2d(d["k_lr"], ws_kl, ug.UG_LR), "rope k_lr")
-        if ev is not None:
-            ev[0].record(stream)
-        if vo_raster:
-            chk(plan.hier_local_attn_fwd_vo_raster(ws_q, ws_k, d["v_hr"], ws_ql, ws_kl,
-                                                   d["v_lr"] if L else None, o_hr, o_lr, lse),
-                "attention")
-        else:
-            chk(plan.hier_local_attn_fwd(ws_q, ws_k, ws_v, ws_ql, ws_kl,
-                                         d["v_lr"] if L else None, ws_o, o_lr, lse), "attention")
-        if ev is not None:
-            ev[1].record(stream)
-        if not vo_raster:
-            chk(plan.unpermute(ws_o, o_hr), "unpermute")
-
-    launches_per_step = 2 + (2 if L else 0) + 1 + (0 if vo_raster else 2)
-    flops = useful_flops(wl)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    st = plan.check_error()
-    if st != ug.UG_OK:
-        raise ug.UgError(st, "warm-up")
-
-    clocks = ClockSampler(local) if rank == 0 else None
-    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize(dev)
-    t0.record(stream)
-    for i in range(args.steps):
-        step(attn_ev[i])
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    clk = clocks.stop() if clocks else None
-    st = plan.check_error()
-    if st != ug.UG_OK:
-        raise ug.UgError(st, "timed steps")
-    sec = t0.elapsed_time(t1) / 1e3 / args.steps
-    attn_sec = sum(a.elapsed_time(b) for a, b in attn_ev) / 1e3 / args.steps
-    sec_max = reduce_max(sec, dev)
-    attn_max = reduce_max(attn_sec, dev)
+    runner, rec = layer_record(args, wl, d, dev, stream, rank, local)
+    plan, o_hr, o_lr, lse, ws = runner.plan, runner.o_hr, runner.o_lr, runner.lse, runner.ws
+    flops = runner.flops
+    sec_max = rec["ms_per_layer"] / 1e3
+    attn_max = rec["attn_ms"] / 1e3
 
     # End to end through the public API: every step copies its inputs from
     # pinned host memory to the device, runs ug_layer_fwd and copies its
@@ -382,9 +549,9 @@ def run_ug(args, wl, world, rank, local):
         in_ready[k].record(s_in)
         stream.wait_event(in_ready[k])
         stream.wait_event(out_free[k])
-        chk(plan.layer_fwd(bi["q_hr"], bi["k_hr"], bi["v_hr"], bi["q_lr"] if L else None,
-                           bi["k_lr"] if L else None, bi["v_lr"] if L else None, oh, ol, lse,
-                           ws, stream), "ug_layer_fwd")
+        _chk(plan.layer_fwd(bi["q_hr"], bi["k_hr"], bi["v_hr"], bi["q_lr"] if L else None,
+                            bi["k_lr"] if L else None, bi["v_lr"] if L else None, oh, ol, lse,
+                            ws, stream), "ug_layer_fwd")
         in_free[k].record(stream)
         out_ready[k].record(stream)
         s_out.wait_event(out_ready[k])
@@ -411,9 +578,30 @@ def run_ug(args, wl, world, rank, local):
     torch.cuda.synchronize(dev)
     barrier()
     e2e_sec = reduce_max(e0.elapsed_time(e1) / 1e3 / args.e2e_steps, dev)
+    del bufs, outs, host_out
+
+    # The layer's backward pass on the same inputs, and the other configs,
+    # timed in the same run (every rank takes the same steps).
+    bwd = None
+    if not args.no_backward:
+        bwd = backward_record(args, wl, d, runner, dev, stream, rank, local)
+    runner.close()
+    del runner, d, pinned
+    torch.cuda.empty_cache()
+    per_config = {}
+    for name in [c for c in args.per_config.split(",") if c and c != wl.name]:
+        pwl = workloads.get(name)
+        pd = workloads.make_inputs_on_device(pwl, seed=rank, device=dev)
+        pd.pop("head_scale", None)
+        steps = max(args.steps, 200) if name in ("tiny", "2K") else args.steps
+        pr, prec = layer_record(args, pwl, pd, dev, stream, rank, local, steps=steps)
+        prec["inputs"] = "drawn on the device (seeded CUDA generator, same distributions)"
+        per_config[name] = prec
+        pr.close()
+        del pr, pd
+        torch.cuda.empty_cache()
 
     if rank == 0:
-        pk, pk_src = peaks()
         achieved = flops / attn_max / 1e12
         line = {
             "metric": METRIC,
@@ -435,31 +623,24 @@ def run_ug(args, wl, world, rank, local):
                 "lowres_grid": [wl.lr_h, wl.lr_w], "rho": wl.rho,
                 "heads": wl.heads, "head_dim": wl.head_dim,
                 "useful_flop_per_layer": flops,
-                "l2": "inputs larger than L2 (each high-res tensor %.0f MB > 126 MB), no flush"
-                      % (hr_bytes / 1e6),
+                "l2": rec["l2"],
                 "parallelism": f"independent layer per GPU x{world}",
             },
             "attn_ms": attn_max * 1e3,
             "attn_tflops": achieved,
-            "roofline": {
-                "bound": "tensor",
-                "achieved": achieved,
-                "peak": pk["bf16_tflops_sustained"],
-                "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_tflops_sustained"],
-                "traffic": attn_traffic_bytes(wl.name),
-                "peak_source": f"{pk_src} bf16 cuBLAS, sustained (kernel timed inside a long step loop)",
-                "frac_of_burst_peak": achieved / pk["bf16_tflops"],
-            },
+            "roofline": rec["roofline"],
             "e2e": {"value": aggregate(flops, world, e2e_sec) / 1e12, "unit": "TFLOP/s",
                     "ms_per_step": e2e_sec * 1e3,
                     "how": "ug_layer_fwd per step with its host-to-device input copy and "
                            "device-to-host output copy (pinned host buffers), steps pipelined "
                            "over copy-in / compute / copy-out streams",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk,
+            "gpu_launches": LayerRunner.launches_of(wl) * args.steps,
+            "clocks": rec["clocks"],
+            "per_config": per_config,
         }
+        if bwd is not None:
+            line["backward"] = bwd
         if not args.no_cpu_baseline and world == 1:
             arm = OracleArm(wl, rows_hr=48, rows_lr=8, heads=range(wl.heads))
             c0 = time.perf_counter()
@@ -467,18 +648,17 @@ def run_ug(args, wl, world, rank, local):
             cdt = time.perf_counter() - c0
             line["cpu_baseline"] = {
                 "value": arm.flops / cdt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
-                "kind": "oracle",
+                "nproc": cpu_cores(), "kind": "oracle",
                 "sample": (f"{len(arm.rows)} query rows x {wl.heads} heads of the {wl.name} "
                            f"layer (RoPE of every key included), fp64 numpy, {cdt:.1f} s"),
             }
         print(json.dumps(line), flush=True)
-    plan.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
 
 
-def run_backward(args, wl, world, rank, local):
+class BackwardRunner:
     """The layer's backward pass: gradients w.r.t. the raster q, k, v given
     the forward's outputs and lse.  A step recomputes the window-first
     rotated operands (5 permutes, 2 of them with RoPE; RoPE of the global q,
@@ -486,80 +666,94 @@ def run_backward(args, wl, world, rank, local):
     events) and maps dq, dk back with the transposed RoPE and the inverse
     permutation.  Useful FLOPs: 2.5 x the forward's (five products per
     visible pair: S, dP, dQ, dK, dV, against the forward's two)."""
+
+    def __init__(self, wl, d, plan, o_hr, o_lr, lse, dev):
+        from block_sparse_local_raster_b200 import ug
+        self.ug, self.wl, self.d, self.plan = ug, wl, d, plan
+        self.o_hr, self.o_lr, self.lse = o_hr, o_lr, lse
+        L = self.L = wl.n_lr
+        lr = self.lr = lambda n: d[n] if L else None
+        e = lambda t: torch.empty_like(t) if t is not None else None
+        self.wf = {n: torch.empty_like(d["q_hr"]) for n in ("q", "k", "v", "o", "do", "dq", "dk", "dv")}
+        self.ql_r, self.kl_r = e(lr("q_lr")), e(lr("k_lr"))
+        self.dq_hr, self.dk_hr, self.dv_hr = e(d["q_hr"]), e(d["k_hr"]), e(d["v_hr"])
+        self.dq_lr, self.dk_lr, self.dv_lr = e(lr("q_lr")), e(lr("k_lr")), e(lr("v_lr"))
+        self.aws = torch.empty(plan.attn_bwd_workspace_bytes(), dtype=torch.uint8, device=dev)
+        self.launches = 5 + (2 if L else 0) + 3 + 3 + (2 if L else 0)
+        self.flops = int(2.5 * useful_flops(wl))
+
+    def step(self, ev=None):
+        ug, d, p, wf, L, lr = self.ug, self.d, self.plan, self.wf, self.L, self.lr
+        _chk(p.permute_rope_window_first(d["q_hr"], wf["q"]), "q")
+        _chk(p.permute_rope_window_first(d["k_hr"], wf["k"]), "k")
+        _chk(p.permute_window_first(d["v_hr"], wf["v"]), "v")
+        _chk(p.permute_window_first(self.o_hr, wf["o"]), "o")
+        _chk(p.permute_window_first(d["do_hr"], wf["do"]), "do")
+        if L:
+            _chk(p.rope_2d(d["q_lr"], self.ql_r, ug.UG_LR), "q_lr")
+            _chk(p.rope_2d(d["k_lr"], self.kl_r, ug.UG_LR), "k_lr")
+        if ev is not None:
+            ev[0].record(torch.cuda.current_stream())
+        _chk(p.hier_local_attn_bwd(wf["q"], wf["k"], wf["v"], self.ql_r, self.kl_r, lr("v_lr"),
+                                   wf["o"], self.o_lr, wf["do"], lr("do_lr"), self.lse, wf["dq"],
+                                   wf["dk"], wf["dv"], self.dq_lr, self.dk_lr, self.dv_lr,
+                                   self.aws), "attention backward")
+        if ev is not None:
+            ev[1].record(torch.cuda.current_stream())
+        _chk(p.unpermute_rope_bwd(wf["dq"], self.dq_hr), "dq")
+        _chk(p.unpermute_rope_bwd(wf["dk"], self.dk_hr), "dk")
+        _chk(p.unpermute(wf["dv"], self.dv_hr), "dv")
+        if L:
+            _chk(p.rope_2d_bwd(self.dq_lr, self.dq_lr, ug.UG_LR), "dq_lr")
+            _chk(p.rope_2d_bwd(self.dk_lr, self.dk_lr, ug.UG_LR), "dk_lr")
+
+
+def backward_record(args, wl, d, fwd, dev, stream, rank, local, steps=None):
+    """Times the layer's backward on inputs d (adds seeded dO) with the
+    forward runner's outputs and lse; returns a record dict."""
+    d = dict(d)
+    d.update(workloads.make_grad_outputs(wl, seed=rank + 1, device=dev))
+    fwd.step()
+    br = BackwardRunner(wl, d, fwd.plan, fwd.o_hr, fwd.o_lr, fwd.lse, dev)
+    steps = steps or args.steps
+    flush = 0 if fwd.hr_bytes > L2_BYTES else 2 * L2_BYTES
+    sec, attn, clk = time_steps(br.step, steps, max(3, min(args.warmup, 5)), dev, stream, rank,
+                                local, flush)
+    _chk(fwd.plan.check_error(), "backward timed steps")
+    ach = br.flops / attn / 1e12
+    return {
+        "metric": "useful attention-backward TFLOP/s & ms per layer backward",
+        "workload": wl.name, "steps": steps, "ms_per_layer_backward": sec * 1e3,
+        "layer_backward_tflops": br.flops / sec / 1e12, "attn_bwd_ms": attn * 1e3,
+        "attn_bwd_tflops": ach, "useful_flop_per_backward": br.flops,
+        "gpu_launches_per_step": br.launches,
+        "roofline": tensor_roofline(ach, attn * steps, clk,
+                                    note="7 products executed per visible pair, 5 counted"),
+        "clocks": clk,
+    }
+
+
+def run_backward(args, wl, world, rank, local):
+    """--op backward: the layer's backward pass alone, with its own end to
+    end through ug_layer_bwd and a CPU-oracle baseline."""
     from block_sparse_local_raster_b200 import ug
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     init_dist("nccl", world)
     stream = torch.cuda.current_stream(dev)
-    plan = ug.Plan(**wl.geom_dict())
     x = workloads.make_inputs(wl, seed=rank)
     x.pop("head_scale", None)
     x.update(workloads.make_grad_outputs(wl, seed=rank + 1))
     d = {k: v.to(dev) for k, v in x.items()}
     L = wl.n_lr
     lr = lambda n: d[n] if L else None
-    o_hr, o_lr, lse = ug.layer_forward(plan, d["q_hr"], d["k_hr"], d["v_hr"], lr("q_lr"),
-                                       lr("k_lr"), lr("v_lr"))
-    B, N, H, Dh = d["q_hr"].shape
-    e = lambda t: torch.empty_like(t) if t is not None else None
-    wf = {n: torch.empty_like(d["q_hr"]) for n in ("q", "k", "v", "o", "do", "dq", "dk", "dv")}
-    ql_r, kl_r = e(lr("q_lr")), e(lr("k_lr"))
-    dq_hr, dk_hr, dv_hr = e(d["q_hr"]), e(d["k_hr"]), e(d["v_hr"])
-    dq_lr, dk_lr, dv_lr = e(lr("q_lr")), e(lr("k_lr")), e(lr("v_lr"))
-    aws = torch.empty(plan.attn_bwd_workspace_bytes(), dtype=torch.uint8, device=dev)
-
-    def chk(st, what):
-        if st != ug.UG_OK:
-            raise ug.UgError(st, what)
-
-    def step(ev=None):
-        chk(plan.permute_rope_window_first(d["q_hr"], wf["q"]), "q")
-        chk(plan.permute_rope_window_first(d["k_hr"], wf["k"]), "k")
-        chk(plan.permute_window_first(d["v_hr"], wf["v"]), "v")
-        chk(plan.permute_window_first(o_hr, wf["o"]), "o")
-        chk(plan.permute_window_first(d["do_hr"], wf["do"]), "do")
-        if L:
-            chk(plan.rope_2d(d["q_lr"], ql_r, ug.UG_LR), "q_lr")
-            chk(plan.rope_2d(d["k_lr"], kl_r, ug.UG_LR), "k_lr")
-        if ev is not None:
-            ev[0].record(stream)
-        chk(plan.hier_local_attn_bwd(wf["q"], wf["k"], wf["v"], ql_r, kl_r, lr("v_lr"), wf["o"],
-                                     o_lr, wf["do"], lr("do_lr"), lse, wf["dq"], wf["dk"],
-                                     wf["dv"], dq_lr, dk_lr, dv_lr, aws), "attention backward")
-        if ev is not None:
-            ev[1].record(stream)
-        chk(plan.unpermute_rope_bwd(wf["dq"], dq_hr), "dq")
-        chk(plan.unpermute_rope_bwd(wf["dk"], dk_hr), "dk")
-        chk(plan.unpermute(wf["dv"], dv_hr), "dv")
-        if L:
-            chk(plan.rope_2d_bwd(dq_lr, dq_lr, ug.UG_LR), "dq_lr")
-            chk(plan.rope_2d_bwd(dk_lr, dk_lr, ug.UG_LR), "dk_lr")
-
-    launches = 5 + (2 if L else 0) + 3 + 3 + (2 if L else 0)
-    flops = int(2.5 * useful_flops(wl))
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    chk(plan.check_error(), "warm-up")
-    clocks = ClockSampler(local) if rank == 0 else None
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize(dev)
-    t0.record(stream)
-    for i in range(args.steps):
-        step(ev[i])
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    clk = clocks.stop() if clocks else None
-    chk(plan.check_error(), "timed steps")
-    sec = reduce_max(t0.elapsed_time(t1) / 1e3 / args.steps, dev)
-    attn = reduce_max(sum(a.elapsed_time(b) for a, b in ev) / 1e3 / args.steps, dev)
+    fwd = LayerRunner(wl, d, dev, stream)
+    fwd.step()
+    br = BackwardRunner(wl, d, fwd.plan, fwd.o_hr, fwd.o_lr, fwd.lse, dev)
+    flush = 0 if fwd.hr_bytes > L2_BYTES else 2 * L2_BYTES
+    sec, attn, clk = time_steps(br.step, args.steps, args.warmup, dev, stream, rank, local, flush)
+    plan, o_hr, o_lr, lse = fwd.plan, fwd.o_hr, fwd.o_lr, fwd.lse
+    _chk(plan.check_error(), "timed steps")
     # end to end: inputs (q, k, v, o, lse, do) from pinned host memory, the
     # gradients back to pinned host memory, through ug_layer_bwd
     ws = torch.empty(plan.layer_bwd_workspace_bytes(), dtype=torch.uint8, device=dev)
@@ -568,7 +762,8 @@ def run_backward(args, wl, world, rank, local):
     if L:
         host_in["o_lr"] = o_lr.cpu().pin_memory()
     dev_in = {"o_hr": o_hr, "lse": lse, **({"o_lr": o_lr} if L else {}), **d}
-    grads = [t for t in (dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr) if t is not None]
+    grads = [t for t in (br.dq_hr, br.dk_hr, br.dv_hr, br.dq_lr, br.dk_lr, br.dv_lr)
+             if t is not None]
     host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in grads]
     e2e_steps = max(3, min(args.e2e_steps, args.steps))
     torch.cuda.synchronize(dev)
@@ -577,16 +772,16 @@ def run_backward(args, wl, world, rank, local):
     for _ in range(e2e_steps):
         for k, v in host_in.items():
             dev_in[k].copy_(v, non_blocking=True)
-        chk(plan.layer_bwd(d["q_hr"], d["k_hr"], d["v_hr"], lr("q_lr"), lr("k_lr"), lr("v_lr"),
-                           o_hr, o_lr, lse, d["do_hr"], lr("do_lr"), dq_hr, dk_hr, dv_hr, dq_lr,
-                           dk_lr, dv_lr, ws, stream), "ug_layer_bwd")
+        _chk(plan.layer_bwd(d["q_hr"], d["k_hr"], d["v_hr"], lr("q_lr"), lr("k_lr"), lr("v_lr"),
+                            o_hr, o_lr, lse, d["do_hr"], lr("do_lr"), br.dq_hr, br.dk_hr,
+                            br.dv_hr, br.dq_lr, br.dk_lr, br.dv_lr, ws, stream), "ug_layer_bwd")
         for h, t in zip(host_out, grads):
             h.copy_(t, non_blocking=True)
     a1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_sec = reduce_max(a0.elapsed_time(a1) / 1e3 / e2e_steps, dev)
+    flops = br.flops
     if rank == 0:
-        pk, src = peaks()
         ach = flops / attn / 1e12
         line = {
             "metric": "useful attention-backward TFLOP/s & ms per layer backward", "op": "backward",
@@ -596,24 +791,22 @@ def run_backward(args, wl, world, rank, local):
             "data": "synthetic",
             "config": {"workload": wl.name, "useful_flop_per_backward": flops,
                        "l2": ("inputs larger than L2 (each high-res tensor %.0f MB), no flush"
-                              if d["q_hr"].numel() * 2 > L2_BYTES else
-                              "inputs smaller than L2 (%.0f MB per high-res tensor), no flush")
-                             % (d["q_hr"].numel() * 2 / 1e6)},
+                              if not flush else
+                              "inputs smaller than L2 (%.0f MB per high-res tensor), flushed "
+                              "between steps") % (d["q_hr"].numel() * 2 / 1e6)},
             "attn_bwd_ms": attn * 1e3, "attn_bwd_tflops": ach,
-            "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops_sustained"],
-                         "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops_sustained"],
-                         "traffic": None, "peak_source": src + " (sustained)",
-                         "executed_products_per_pair": 7},
+            "roofline": tensor_roofline(ach, attn * args.steps, clk,
+                                        note="7 products executed per visible pair, 5 counted"),
             "e2e": {"value": aggregate(flops, world, e2e_sec) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": sum(v.numel() * v.element_size()
                                               for v in host_in.values()),
                     "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in grads)},
-            "gpu_launches": launches * args.steps, "clocks": clk,
+            "gpu_launches": br.launches * args.steps, "clocks": clk,
         }
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = backward_cpu_baseline(wl, x)
         print(json.dumps(line), flush=True)
-    plan.close()
+    fwd.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -637,7 +830,7 @@ def backward_cpu_baseline(wl, x):
     O.layer_backward(bits, bits, g, rows=rows, keys=np.zeros(0, dtype=np.int64))
     cdt = time.perf_counter() - c0
     flops = 2.5 * 4 * g.head_dim * vis
-    return {"value": flops / cdt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+    return {"value": flops / cdt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "nproc": cpu_cores(),
             "kind": "oracle",
             "sample": (f"dq of {rows.size} query rows x 1 head of the {wl.name} layer backward "
                        f"(RoPE of every key included), fp64 numpy, {cdt:.1f} s")}
@@ -729,7 +922,7 @@ def run_warm_start(args, world, rank, local):
             W.warm_start(xs, ns, ws.scale, ws.sharpen, ws.t)
             cdt = time.perf_counter() - c0
             b1 = (xs.size + 2 * ns.size) * 4
-            line["cpu_baseline"] = {"value": b1 / cdt / 1e9, "unit": "GB/s", "cores": cpu_threads(),
+            line["cpu_baseline"] = {"value": b1 / cdt / 1e9, "unit": "GB/s", "cores": cpu_threads(), "nproc": cpu_cores(),
                                     "kind": "oracle",
                                     "sample": f"one plane of the latent, fp64 numpy, {cdt:.2f} s"}
         print(json.dumps(line), flush=True)

@@ -19,6 +19,17 @@ bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
   return pa < pb + nb && pb < pa + na;
 }
 
+// The plan's tables live in the memory of the device that was current when
+// it was created; its kernels must launch there.
+int check_device(const ug_plan* p) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return UG_ERR_CUDA;
+  }
+  return dev == p->device ? UG_OK : UG_ERR_INVALID_ARG;
+}
+
 int64_t hr_bytes(const ug_plan* p) {
   return (int64_t)p->g.batch * p->N * p->g.heads * p->g.head_dim * 2;
 }
@@ -183,6 +194,13 @@ int ug_plan_create(const ug_geom* g, ug_plan** out) {
     const size_t a_ql = (a_kt + p->ktiles.size() * sizeof(KTile) + 255) / 256 * 256;
     const size_t total = a_ql + std::max<size_t>(1, p->qlist.size()) * sizeof(uint32_t);
     if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return UG_ERR_CUDA; }
+    // once per device: kernel attributes, the static scratch's address
+    if ((st = prepare_attention(p->device)) != UG_OK ||
+        (st = prepare_attention_bwd(p->device)) != UG_OK ||
+        (st = prepare_static_scratch(p->device)) != UG_OK) {
+      delete p;
+      return st;
+    }
     if (cudaMalloc(&p->d_mem, total) != cudaSuccess) {
       cudaGetLastError();
       delete p;
@@ -219,8 +237,14 @@ int ug_plan_destroy(ug_plan* p) {
   if (!p) return UG_OK;
   int st = UG_OK;
   if (p->d_mem) {
+    // free on the plan's device, then restore the caller's current device
+    int cur = -1;
+    const bool have_cur = cudaGetDevice(&cur) == cudaSuccess;
+    const bool other = have_cur && cur != p->device;
+    if (other && cudaSetDevice(p->device) != cudaSuccess) st = UG_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) st = UG_ERR_CUDA;
     if (cudaFree(p->d_mem) != cudaSuccess) st = UG_ERR_CUDA;
+    if (other && cudaSetDevice(cur) != cudaSuccess) st = UG_ERR_CUDA;
   }
   delete p;
   return st;
@@ -239,6 +263,7 @@ static int permute_common(const ug_plan* p, const void* src, void* dst, bool inv
   if (!aligned16(src) || !aligned16(dst)) return UG_ERR_ALIGNMENT;
   const int64_t n = hr_bytes(p);
   if (overlap(src, n, dst, n)) return UG_ERR_ALIAS;
+  if (const int st = check_device(p)) return st;
   return launch_permute(p, src, dst, inverse, as_stream(s));
 }
 
@@ -252,6 +277,7 @@ int ug_permute_rope_window_first(const ug_plan* p, const void* src_raster, void*
   if (!aligned16(src_raster) || !aligned16(dst_wf)) return UG_ERR_ALIGNMENT;
   const int64_t n = hr_bytes(p);
   if (overlap(src_raster, n, dst_wf, n)) return UG_ERR_ALIAS;
+  if (const int st = check_device(p)) return st;
   return launch_permute_rope(p, src_raster, dst_wf, as_stream(s));
 }
 
@@ -267,6 +293,7 @@ int ug_rope_2d(const ug_plan* p, const void* x, void* y, int token_set, void* s)
   const int64_t n = token_set == UG_LR ? lr_bytes(p) : hr_bytes(p);
   if (n == 0) return UG_OK;
   if (x != y && overlap(x, n, y, n)) return UG_ERR_ALIAS;
+  if (const int st = check_device(p)) return st;
   return launch_rope(p, x, y, token_set, as_stream(s));
 }
 
@@ -274,12 +301,15 @@ int ug_rope_2d(const ug_plan* p, const void* x, void* y, int token_set, void* s)
 
 namespace {
 
-int attn_fwd_checked(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
-                     const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
-                     void* o_lr, float* lse, bool vo_raster, void* s) {
+// Pointers, alignment and overlaps of a forward call's tensors: inputs
+// q/k/v (high-res and global), outputs o_hr, o_lr and the optional lse.
+int check_fwd_tensors(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+                      const void* q_lr, const void* k_lr, const void* v_lr, const void* o_hr,
+                      const void* o_lr, const float* lse) {
   if (!p || !q_hr || !k_hr || !v_hr || !o_hr) return UG_ERR_INVALID_ARG;
   if (p->L > 0 && (!q_lr || !k_lr || !v_lr || !o_lr)) return UG_ERR_INVALID_ARG;
   if (p->g.head_dim != 64 && p->g.head_dim != 128) return UG_ERR_UNSUPPORTED;
+  if (p->L == 0) q_lr = k_lr = v_lr = o_lr = nullptr;
   const void* ins[6] = {q_hr, k_hr, v_hr, q_lr, k_lr, v_lr};
   for (const void* a : ins)
     if (a && !aligned16(a)) return UG_ERR_ALIGNMENT;
@@ -295,6 +325,15 @@ int attn_fwd_checked(const ug_plan* p, const void* q_hr, const void* k_hr, const
   }
   if (overlap(o_hr, nh, o_lr, nl) || overlap(o_hr, nh, lse, nlse) || overlap(o_lr, nl, lse, nlse))
     return UG_ERR_ALIAS;
+  return UG_OK;
+}
+
+int attn_fwd_checked(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+                     const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
+                     void* o_lr, float* lse, bool vo_raster, void* s) {
+  if (const int st = check_fwd_tensors(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse))
+    return st;
+  if (const int st = check_device(p)) return st;
   return launch_attention(p, q_hr, k_hr, v_hr, p->L ? q_lr : nullptr, p->L ? k_lr : nullptr,
                           p->L ? v_lr : nullptr, o_hr, p->L ? o_lr : nullptr, lse, vo_raster,
                           as_stream(s));
@@ -329,18 +368,20 @@ int64_t ug_layer_workspace_bytes(const ug_plan* p) {
 int ug_layer_fwd(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                  const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr, void* o_lr,
                  float* lse, void* workspace, int64_t workspace_bytes, void* s) {
+  // Every argument check runs here, before the first launch is queued.
   if (!p || !workspace) return UG_ERR_INVALID_ARG;
   if (workspace_bytes < ug_layer_workspace_bytes(p)) return UG_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return UG_ERR_ALIGNMENT;
-  if (!q_hr || !k_hr || !v_hr || !o_hr) return UG_ERR_INVALID_ARG;
-  if (p->L > 0 && (!q_lr || !k_lr || !v_lr || !o_lr)) return UG_ERR_INVALID_ARG;
-  if (p->g.head_dim != 64 && p->g.head_dim != 128) return UG_ERR_UNSUPPORTED;
+  if (const int st = check_fwd_tensors(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse))
+    return st;
   const int64_t ws = ug_layer_workspace_bytes(p);
-  const void* ins[6] = {q_hr, k_hr, v_hr, q_lr, k_lr, v_lr};
   const int64_t nh = hr_bytes(p), nl = lr_bytes(p);
-  const int64_t sizes[6] = {nh, nh, nh, nl, nl, nl};
-  for (int i = 0; i < 6; ++i)
-    if (overlap(workspace, ws, ins[i], sizes[i])) return UG_ERR_ALIAS;
+  const int64_t nlse = lse ? (int64_t)p->g.batch * p->g.heads * (p->N + p->L) * 4 : 0;
+  const void* ts[9] = {q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse};
+  const int64_t sizes[9] = {nh, nh, nh, nl, nl, nl, nh, nl, nlse};
+  for (int i = 0; i < 9; ++i)
+    if (overlap(workspace, ws, ts[i], sizes[i])) return UG_ERR_ALIAS;
+  if (const int st = check_device(p)) return st;
   auto up = [](int64_t n) { return (n + 255) / 256 * 256; };
   char* w = static_cast<char*>(workspace);
   void* q_wf = w;
@@ -349,8 +390,6 @@ int ug_layer_fwd(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   void* o_wf = w + 3 * up(nh);
   void* q_lr_r = w + 4 * up(nh);
   void* k_lr_r = w + 4 * up(nh) + up(nl);
-  if (overlap(workspace, ws, o_hr, nh) || overlap(workspace, ws, o_lr, nl))
-    return UG_ERR_ALIAS;
   int st;
   if ((st = ug_permute_rope_window_first(p, q_hr, q_wf, s)) != UG_OK) return st;
   if ((st = ug_permute_rope_window_first(p, k_hr, k_wf, s)) != UG_OK) return st;
@@ -380,6 +419,7 @@ int ug_rope_2d_bwd(const ug_plan* p, const void* dy, void* dx, int token_set, vo
   const int64_t n = token_set == UG_LR ? lr_bytes(p) : hr_bytes(p);
   if (n == 0) return UG_OK;
   if (dy != dx && overlap(dy, n, dx, n)) return UG_ERR_ALIAS;
+  if (const int st = check_device(p)) return st;
   return launch_rope(p, dy, dx, token_set, as_stream(s), true);
 }
 
@@ -388,6 +428,7 @@ int ug_unpermute_rope_bwd(const ug_plan* p, const void* src_wf, void* dst_raster
   if (!aligned16(src_wf) || !aligned16(dst_raster)) return UG_ERR_ALIGNMENT;
   const int64_t n = hr_bytes(p);
   if (overlap(src_wf, n, dst_raster, n)) return UG_ERR_ALIAS;
+  if (const int st = check_device(p)) return st;
   return launch_permute_rope(p, src_wf, dst_raster, as_stream(s), true);
 }
 
@@ -430,6 +471,7 @@ int ug_hier_local_attn_bwd(const ug_plan* p, const void* q_hr, const void* k_hr,
     for (int j = i + 1; j < 7; ++j)
       if (overlap(w[i], wn[i], w[j], wn[j])) return UG_ERR_ALIAS;
   }
+  if (const int st = check_device(p)) return st;
   return launch_attention_bwd(p, q_hr, k_hr, v_hr, lr ? q_lr : nullptr, lr ? k_lr : nullptr,
                               lr ? v_lr : nullptr, o_hr, lr ? o_lr : nullptr, do_hr,
                               lr ? do_lr : nullptr, lse, dq_hr, dk_hr, dv_hr,
@@ -466,6 +508,23 @@ int ug_layer_bwd(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
     if (overlap(workspace, ws, ins[i], i < 5 ? nh : nl)) return UG_ERR_ALIAS;
   for (int i = 0; i < 6; ++i)
     if (overlap(workspace, ws, outs[i], i < 3 ? nh : nl)) return UG_ERR_ALIAS;
+  // the gradients are disjoint from every input and from each other
+  const int64_t nlse = (int64_t)p->g.batch * p->g.heads * (p->N + p->L) * 4;
+  if (overlap(workspace, ws, lse, nlse)) return UG_ERR_ALIAS;
+  for (int i = 0; i < 6; ++i) {
+    const int64_t ni = i < 3 ? nh : nl;
+    for (int j = 0; j < 10; ++j)
+      if (overlap(outs[i], ni, ins[j], j < 5 ? nh : nl)) return UG_ERR_ALIAS;
+    if (overlap(outs[i], ni, lse, nlse)) return UG_ERR_ALIAS;
+    for (int j = i + 1; j < 6; ++j)
+      if (overlap(outs[i], ni, outs[j], j < 3 ? nh : nl)) return UG_ERR_ALIAS;
+  }
+  for (int i = 0; i < 10; ++i)
+    if ((i < 5 || lr) && !aligned16(ins[i])) return UG_ERR_ALIGNMENT;
+  for (int i = 0; i < 6; ++i)
+    if ((i < 3 || lr) && !aligned16(outs[i])) return UG_ERR_ALIGNMENT;
+  if (!aligned16(lse)) return UG_ERR_ALIGNMENT;
+  if (const int st = check_device(p)) return st;
   auto up = [](int64_t n) { return (n + 255) / 256 * 256; };
   char* w = static_cast<char*>(workspace);
   void* q_wf = w;
@@ -530,6 +589,7 @@ int ug_warm_start(const ug_warm_start_params* q, const float* x_lr, const float*
 
 int ug_check_error(const ug_plan* p, void* s) {
   if (!p) return UG_ERR_INVALID_ARG;
+  if (const int st = check_device(p)) return st;
   if (cudaStreamSynchronize(as_stream(s)) != cudaSuccess) return UG_ERR_CUDA;
   int h = 0;
   if (cudaMemcpy(&h, p->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)

@@ -47,6 +47,7 @@
 #include <cuda_bf16.h>
 
 #include "ug_internal.h"
+#include "ug_per_device.h"
 #include "ug_tc.cuh"
 
 namespace ug {
@@ -476,20 +477,31 @@ int launch_d(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v
   P.grid_w = p->g.grid_w;
   P.win_h = p->g.win_h;
   P.win_w = p->g.win_w;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(hier_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Layout<D>::kAlloc) != cudaSuccess)
-      return UG_ERR_CUDA;
-    attr_set = true;
-  }
+  if (const int pst = prepare_attention(p->device)) return pst;
   const dim3 grid((unsigned)p->qtiles.size(), (unsigned)H, (unsigned)B);
   hier_attn_kernel<D><<<grid, kThreads, Layout<D>::kAlloc, st>>>(m[0], m[1], m[2], m[3], m[4],
                                                                   m[5], P);
   return cudaGetLastError() == cudaSuccess ? UG_OK : UG_ERR_CUDA;
 }
 
+PerDevice<char> g_attn_ready;
+
 }  // namespace
+
+// The kernels need more than 48 KB of dynamic shared memory, an opt-in that
+// is per device; done once per device (ug_plan_create calls this).
+int prepare_attention(int device) {
+  return g_attn_ready.get(device, [](char&) {
+    const bool ok = cudaFuncSetAttribute(hier_attn_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Layout<128>::kAlloc) == cudaSuccess &&
+                    cudaFuncSetAttribute(hier_attn_kernel<64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Layout<64>::kAlloc) == cudaSuccess;
+    if (!ok) cudaGetLastError();
+    return ok ? UG_OK : UG_ERR_CUDA;
+  });
+}
 
 int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                      const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,

@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 
 #include "ug_internal.h"
+#include "ug_per_device.h"
 #include "ug_tc.cuh"
 
 namespace ug {
@@ -856,15 +857,7 @@ int launch_bwd_d(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   P.heads = H;
   P.scale = p->scale;
   P.scale_log2 = p->scale * kLog2e;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DqLayout<D>::kAlloc) != cudaSuccess ||
-        cudaFuncSetAttribute(dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DkvLayout<D>::kAlloc) != cudaSuccess)
-      return UG_ERR_CUDA;
-    attr_set = true;
-  }
+  if (const int pst = prepare_attention_bwd(p->device)) return pst;
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device);
   const int64_t rows = B * (p->N + p->L);
@@ -883,7 +876,27 @@ int launch_bwd_d(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   return cudaGetLastError() == cudaSuccess ? UG_OK : UG_ERR_CUDA;
 }
 
+PerDevice<char> g_bwd_ready;
+
 }  // namespace
+
+// The dQ and dK/dV kernels need more than 48 KB of dynamic shared memory, an
+// opt-in that is per device; done once per device (ug_plan_create calls this).
+int prepare_attention_bwd(int device) {
+  return g_bwd_ready.get(device, [](char&) {
+    const bool ok =
+        cudaFuncSetAttribute(dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DqLayout<128>::kAlloc) == cudaSuccess &&
+        cudaFuncSetAttribute(dkv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkvLayout<128>::kAlloc) == cudaSuccess &&
+        cudaFuncSetAttribute(dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DqLayout<64>::kAlloc) == cudaSuccess &&
+        cudaFuncSetAttribute(dkv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkvLayout<64>::kAlloc) == cudaSuccess;
+    if (!ok) cudaGetLastError();
+    return ok ? UG_OK : UG_ERR_CUDA;
+  });
+}
 
 int launch_attention_bwd(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                          const void* q_lr, const void* k_lr, const void* v_lr, const void* o_hr,

@@ -120,6 +120,12 @@ int launch_warm_start(const ug_warm_start_params* p, const float* x_lr, const fl
 int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                      const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
                      void* o_lr, float* lse, bool vo_raster, cudaStream_t s);
+// Per-device set-up, done once per device and run by ug_plan_create with the
+// plan's device current: the attention kernels' shared-memory opt-in, and the
+// device address of the static scratch of ug_layer_fwd_static_scratch.
+int prepare_attention(int device);
+int prepare_attention_bwd(int device);
+int prepare_static_scratch(int device);
 // Whether a 128-key tile is always 128 / win_w whole rows of one window, so
 // that raster-order V can be read tile by tile.
 bool vo_raster_supported(const ug_geom& g);

@@ -11,41 +11,41 @@
 // intermediates live in g_layer_scratch below, which every GPU that loads
 // this library holds until the process exits.
 #include <cstdint>
-#include <mutex>
 
 #include "ug_internal.h"
+#include "ug_per_device.h"
 
 namespace {
 
 constexpr int64_t kScratchBytes = UG_STATIC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 // Device-side scratch.  In host code this name is only a host-side stand-in
 // for the symbol, not a device address; the device address comes from
 // cudaGetSymbolAddress below, per device.
 __device__ __align__(256) unsigned char g_layer_scratch[kScratchBytes];
 
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices];  // device address of g_layer_scratch per device
-
-// Device address of the scratch on the current device; looked up on the
-// first call for that device (with that device current) and cached.
-int scratch_on_current_device(int device, void** out) {
-  if (device < 0 || device >= kMaxDevices) return UG_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[device]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_layer_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();
-      return UG_ERR_CUDA;
-    }
-    g_scratch_ptr[device] = p;
-  }
-  *out = g_scratch_ptr[device];
-  return UG_OK;
-}
+// Device address of g_layer_scratch, per device.
+ug::PerDevice<void*> g_scratch_ptr;
 
 }  // namespace
+
+namespace ug {
+
+// Looks up the scratch's device address with `device` current and caches it.
+// ug_plan_create calls this during set-up: under lazy module loading the
+// lookup is what loads this module (and places the array), so it happens
+// there, not on the allocation-free call path.
+int prepare_static_scratch(int device) {
+  return g_scratch_ptr.get(device, [](void*& ptr) {
+    if (cudaGetSymbolAddress(&ptr, g_layer_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return (int)UG_ERR_CUDA;
+    }
+    return (int)UG_OK;
+  });
+}
+
+}  // namespace ug
 
 extern "C" int ug_layer_fwd_static_scratch(const ug_plan* p, const void* q_hr, const void* k_hr,
                                            const void* v_hr, const void* q_lr, const void* k_lr,
@@ -58,8 +58,8 @@ extern "C" int ug_layer_fwd_static_scratch(const ug_plan* p, const void* q_hr, c
   if (cudaGetDevice(&dev) != cudaSuccess) return UG_ERR_CUDA;
   if (dev != p->device) return UG_ERR_INVALID_ARG;
   void* scratch = nullptr;
-  const int st = scratch_on_current_device(dev, &scratch);
-  if (st != UG_OK) return st;
+  const int st = g_scratch_ptr.get(dev, [](void*&) { return (int)UG_ERR_CUDA; }, &scratch);
+  if (st != UG_OK) return st;  // set-up (ug_plan_create on this device) has not succeeded
   // Every byte of the scratch that the layer reads it first writes in the
   // same call, so nothing needs clearing between calls.
   return ug_layer_fwd(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, scratch, need,

@@ -161,6 +161,31 @@ def make_inputs(wl: Workload, seed: int = 0,
     return out
 
 
+def make_inputs_on_device(wl: Workload, seed: int, device) -> Dict[str, torch.Tensor]:
+    """The same distributions as make_inputs, drawn on the device by a seeded
+    CUDA generator (a different random stream, so different values): for
+    timing runs at sizes where the CPU draw takes minutes (8K: 805 M normals
+    per tensor).  Parity tests use make_inputs."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    shp_hr = (wl.batch, wl.n_hr, wl.heads, wl.head_dim)
+    shp_lr = (wl.batch, wl.n_lr, wl.heads, wl.head_dim)
+    out: Dict[str, torch.Tensor] = {}
+    s = None
+    if wl.head_scale:
+        s = torch.empty((3, wl.heads), dtype=torch.float32, device=device).uniform_(
+            0.5, 2.0, generator=g)
+    for name, shp in (("q_hr", shp_hr), ("k_hr", shp_hr), ("v_hr", shp_hr),
+                      ("q_lr", shp_lr), ("k_lr", shp_lr), ("v_lr", shp_lr)):
+        t = torch.randn(shp, generator=g, dtype=torch.float32, device=device)
+        if s is not None:
+            t.mul_(s["qkv".index(name[0])].view(1, 1, wl.heads, 1))
+        out[name] = t.to(torch.bfloat16).contiguous()
+        del t
+    if s is not None:
+        out["head_scale"] = s
+    return out
+
+
 def make_grad_outputs(wl: Workload, seed: int = 1,
                       device: Optional[str] = None) -> Dict[str, torch.Tensor]:
     """Seeded output gradients for the backward pass: do_hr [B, N, h, d] and

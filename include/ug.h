@@ -37,6 +37,11 @@
  *     ug_plan_destroy frees it.
  *   - Every call returns a ug_status; no C++ exception crosses the ABI.
  *     Argument errors are reported before any work is queued.
+ *   - A plan belongs to the device that was current when it was created:
+ *     every call taking a plan must run with that device current
+ *     (UG_ERR_INVALID_ARG otherwise), because the plan's tables live in that
+ *     device's memory.  Plans on several devices of one process, and calls
+ *     from several host threads, are supported.
  */
 #ifndef UG_H_
 #define UG_H_
@@ -270,8 +275,10 @@ int ug_layer_fwd(const ug_plan* plan, const void* q_hr, const void* k_hr, const 
  *   - UG_ERR_UNSUPPORTED, before any work is queued, when the plan's
  *     ug_layer_workspace_bytes exceeds UG_STATIC_SCRATCH_BYTES;
  *     UG_ERR_INVALID_ARG when the plan's device is not the current device.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
+ *   - ug_plan_create looks up the array's device address
+ *     (cudaGetSymbolAddress) once per device, with the plan's device
+ *     current; that lookup is also what loads the array onto the device, so
+ *     it happens at set-up and not on this call's path.  Create the plan
  *     before any stream capture.
  *   - Every call shares the one array, which keeps the last call's contents.
  *     Nothing in it needs clearing (each call writes what it reads), but calls

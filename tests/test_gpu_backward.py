@@ -54,11 +54,15 @@ def joint_grads(grads, wl, heads=None):
 
 
 def check(got, ref, bound, what):
-    excess = np.abs(got - ref) - bound
+    """Every element within its derived bound; prints the worst ratio
+    |error| / bound (the headroom actually left)."""
+    err = np.abs(got - ref)
+    excess = err - bound
     worst = np.unravel_index(np.argmax(excess), excess.shape)
-    assert excess.max() <= 0, (what, float(excess.max()), float(np.abs(got - ref)[worst]),
+    print(f"{what}: max |err| {err.max():.3g}, worst |err| / bound {(err / bound).max():.3f}")
+    assert excess.max() <= 0, (what, float(excess.max()), float(err[worst]),
                                float(bound[worst]), worst)
-    return float(np.abs(got - ref).max())
+    return float(err.max())
 
 
 @pytest.mark.parametrize("name", SMALL)
@@ -117,8 +121,8 @@ def test_attention_backward_sampled_full_size(name):
     mag = lambda a, b_: a.double().abs().sum(1) + b_.double().abs().sum(1)
     dk_hr, dv_hr, dk_lr, dv_lr = grads[1], grads[2], grads[4], grads[5]
     do_sum = tot(x["do_hr"].to(DEV), x["do_lr"].to(DEV))
-    assert bool(((tot(dv_hr, dv_lr) - do_sum).abs() <= 2 * U * mag(dv_hr, dv_lr) + 1e-3).all())
-    assert bool((tot(dk_hr, dk_lr).abs() <= 4 * U * mag(dk_hr, dk_lr) + 1e-3).all())
+    assert bool(((tot(dv_hr, dv_lr) - do_sum).abs() <= U * mag(dv_hr, dv_lr) + 1e-3).all())
+    assert bool((tot(dk_hr, dk_lr).abs() <= 2 * U * mag(dk_hr, dk_lr) + 1e-3).all())
 
 
 SETS = [(ug.UG_HR_WINDOW_FIRST, O.HR_WINDOW_FIRST), (ug.UG_HR_RASTER, O.HR_RASTER),

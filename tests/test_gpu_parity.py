@@ -135,8 +135,10 @@ def check_rows(wl, g, o_hr, o_lr, lse, ref_o, ref_lse, rows, vscale=None):
     got = np.concatenate([f64(o_hr[:, torch.from_numpy(hr)]),
                           f64(o_lr[:, torch.from_numpy(lr)]) if lr.size else
                           np.zeros((wl.batch, 0, wl.heads, wl.head_dim))], axis=1)
-    mx, mean = err_stats(got, ref_o, vscale)
+    mx, mean, raw, raw_lim = err_stats(got, ref_o, vscale)
+    print(f"max-abs {mx:.3g} (raw {raw:.3g}, raw bound {raw_lim:.3g}), mean-abs {mean:.3g}")
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+    assert raw <= raw_lim, (raw, raw_lim)
     lse_got = lse.cpu().numpy()[:, :, np.concatenate([hr, N + lr])]
     assert np.abs(lse_got - ref_lse).max() <= LSE_ABS, np.abs(lse_got - ref_lse).max()
     return mx, mean
@@ -238,8 +240,10 @@ def test_layer_end_to_end(name):
                           f64(o_lr[:, torch.from_numpy(lrr)]) if lrr.size else
                           np.zeros((wl.batch, 0, wl.heads, wl.head_dim))], axis=1)
     vs = x["head_scale"][2].numpy() if "head_scale" in x else None
-    mx, mean = err_stats(got, ref_o, vs)
+    mx, mean, raw, raw_lim = err_stats(got, ref_o, vs)
+    print(f"max-abs {mx:.3g} (raw {raw:.3g}, raw bound {raw_lim:.3g}), mean-abs {mean:.3g}")
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+    assert raw <= raw_lim, (raw, raw_lim)
     lse_got = lse.cpu().numpy()[:, :, lse_rows]
     assert np.abs(lse_got - ref_lse).max() <= LSE_ABS
 

@@ -64,3 +64,22 @@ def test_overflow_and_zero():
     assert O.f64_to_bf16(np.array([-0.0]))[0] == 0x8000
     assert O.f64_to_bf16(np.array([2.0 ** -134]))[0] == 0  # half the smallest subnormal: tie -> 0
     assert O.f64_to_bf16(np.array([2.0 ** -134 * 1.5]))[0] == 1
+
+
+def test_half_ulp_bound_of_the_parity_checks():
+    """parity.half_ulp_bf16 is the most that rounding to bf16 moves a value:
+    torch's (single) rounding of 200k random fp32 values from many binades
+    stays within it, and values exactly halfway between two bf16 neighbours
+    reach it."""
+    from parity import half_ulp_bf16
+    rng = np.random.default_rng(3)
+    x32 = (rng.standard_normal(200_000) * np.exp2(rng.integers(-20, 20, 200_000)))
+    x32 = x32.astype(np.float32)
+    x = x32.astype(np.float64)
+    r = torch.from_numpy(x32).to(torch.bfloat16).double().numpy()
+    assert (np.abs(r - x) <= half_ulp_bf16(x)).all()
+    # midpoints between consecutive bf16 values in [1, 2): ulp 2^-7
+    k = np.arange(128)
+    mid = 1.0 + (k + 0.5) * 2.0 ** -7
+    rm = torch.from_numpy(mid.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(np.abs(rm - mid), half_ulp_bf16(mid))
