@@ -661,10 +661,11 @@ def run_ug(args, wl, world, rank, local):
 class BackwardRunner:
     """The layer's backward pass: gradients w.r.t. the raster q, k, v given
     the forward's outputs and lse.  A step recomputes the window-first
-    rotated operands (5 permutes, 2 of them with RoPE; RoPE of the global q,
-    k), runs the attention backward (D, dQ, dK/dV kernels; timed alone with
-    events) and maps dq, dk back with the transposed RoPE and the inverse
-    permutation.  Useful FLOPs: 2.5 x the forward's (five products per
+    rotated q and k (2 fused permutes with RoPE; RoPE of the global q, k),
+    runs the attention backward (D, dQ, dK/dV kernels; timed alone with
+    events; v, o, dO read and dv written in raster order where 128-row tiles
+    are whole window rows, else 3 more permutes and 1 unpermute) and maps dq,
+    dk back with the transposed RoPE and the inverse permutation.  Useful FLOPs: 2.5 x the forward's (five products per
     visible pair: S, dP, dQ, dK, dV, against the forward's two)."""
 
     def __init__(self, wl, d, plan, o_hr, o_lr, lse, dev):
@@ -679,30 +680,43 @@ class BackwardRunner:
         self.dq_hr, self.dk_hr, self.dv_hr = e(d["q_hr"]), e(d["k_hr"]), e(d["v_hr"])
         self.dq_lr, self.dk_lr, self.dv_lr = e(lr("q_lr")), e(lr("k_lr")), e(lr("v_lr"))
         self.aws = torch.empty(plan.attn_bwd_workspace_bytes(), dtype=torch.uint8, device=dev)
-        self.launches = 5 + (2 if L else 0) + 3 + 3 + (2 if L else 0)
+        # where 128-row tiles are whole window rows the backward reads v, o, dO
+        # and writes dv in raster order (no permutes of v, o, dO, no unpermute of dv)
+        T = wl.win_h * wl.win_w
+        self.vo_raster = 128 % wl.win_w == 0 and T % 128 == 0
+        self.launches = (2 + (0 if self.vo_raster else 3) + (2 if L else 0) + 3 + 2
+                         + (0 if self.vo_raster else 1) + (2 if L else 0))
         self.flops = int(2.5 * useful_flops(wl))
 
     def step(self, ev=None):
         ug, d, p, wf, L, lr = self.ug, self.d, self.plan, self.wf, self.L, self.lr
         _chk(p.permute_rope_window_first(d["q_hr"], wf["q"]), "q")
         _chk(p.permute_rope_window_first(d["k_hr"], wf["k"]), "k")
-        _chk(p.permute_window_first(d["v_hr"], wf["v"]), "v")
-        _chk(p.permute_window_first(self.o_hr, wf["o"]), "o")
-        _chk(p.permute_window_first(d["do_hr"], wf["do"]), "do")
+        if not self.vo_raster:
+            _chk(p.permute_window_first(d["v_hr"], wf["v"]), "v")
+            _chk(p.permute_window_first(self.o_hr, wf["o"]), "o")
+            _chk(p.permute_window_first(d["do_hr"], wf["do"]), "do")
         if L:
             _chk(p.rope_2d(d["q_lr"], self.ql_r, ug.UG_LR), "q_lr")
             _chk(p.rope_2d(d["k_lr"], self.kl_r, ug.UG_LR), "k_lr")
         if ev is not None:
             ev[0].record(torch.cuda.current_stream())
-        _chk(p.hier_local_attn_bwd(wf["q"], wf["k"], wf["v"], self.ql_r, self.kl_r, lr("v_lr"),
-                                   wf["o"], self.o_lr, wf["do"], lr("do_lr"), self.lse, wf["dq"],
-                                   wf["dk"], wf["dv"], self.dq_lr, self.dk_lr, self.dv_lr,
-                                   self.aws), "attention backward")
+        if self.vo_raster:
+            _chk(p.hier_local_attn_bwd_vo_raster(
+                wf["q"], wf["k"], d["v_hr"], self.ql_r, self.kl_r, lr("v_lr"), self.o_hr,
+                self.o_lr, d["do_hr"], lr("do_lr"), self.lse, wf["dq"], wf["dk"], self.dv_hr,
+                self.dq_lr, self.dk_lr, self.dv_lr, self.aws), "attention backward")
+        else:
+            _chk(p.hier_local_attn_bwd(wf["q"], wf["k"], wf["v"], self.ql_r, self.kl_r,
+                                       lr("v_lr"), wf["o"], self.o_lr, wf["do"], lr("do_lr"),
+                                       self.lse, wf["dq"], wf["dk"], wf["dv"], self.dq_lr,
+                                       self.dk_lr, self.dv_lr, self.aws), "attention backward")
         if ev is not None:
             ev[1].record(torch.cuda.current_stream())
         _chk(p.unpermute_rope_bwd(wf["dq"], self.dq_hr), "dq")
         _chk(p.unpermute_rope_bwd(wf["dk"], self.dk_hr), "dk")
-        _chk(p.unpermute(wf["dv"], self.dv_hr), "dv")
+        if not self.vo_raster:
+            _chk(p.unpermute(wf["dv"], self.dv_hr), "dv")
         if L:
             _chk(p.rope_2d_bwd(self.dq_lr, self.dq_lr, ug.UG_LR), "dq_lr")
             _chk(p.rope_2d_bwd(self.dk_lr, self.dk_lr, ug.UG_LR), "dk_lr")

@@ -181,13 +181,12 @@ int ug_plan_create(const ug_geom* g, ug_plan** out) {
     build_attention_lists(*g, p->nbr_off, p->nbr_idx, p->qtiles, p->kvlist, &p->n_hr_ctas,
                           &p->n_lr_ctas);
     build_backward_lists(*g, p->nbr_off, p->nbr_idx, p->ktiles, p->qlist);
-    std::vector<float> tables32;
-    build_rope_tables(*g, p->rope, tables32);
-    const std::vector<double> tables(tables32.begin(), tables32.end());
+    std::vector<float> tables;
+    build_rope_tables(*g, p->rope, tables);
     // One device block: [err (256 B)] [rope tables] [qtiles] [kvlist] [ktiles] [qlist]
     const size_t a_err = 0;
     const size_t a_rope = 256;
-    const size_t a_qt = (a_rope + tables.size() * sizeof(double) + 255) / 256 * 256;
+    const size_t a_qt = (a_rope + tables.size() * sizeof(float) + 255) / 256 * 256;
     const size_t a_kv = (a_qt + p->qtiles.size() * sizeof(QTile) + 255) / 256 * 256;
     const size_t a_kt = (a_kv + std::max<size_t>(1, p->kvlist.size()) * sizeof(uint32_t) + 255) /
                         256 * 256;
@@ -197,6 +196,7 @@ int ug_plan_create(const ug_geom* g, ug_plan** out) {
     // once per device: kernel attributes, the static scratch's address
     if ((st = prepare_attention(p->device)) != UG_OK ||
         (st = prepare_attention_bwd(p->device)) != UG_OK ||
+        (st = prepare_rope(p->device)) != UG_OK ||
         (st = prepare_static_scratch(p->device)) != UG_OK) {
       delete p;
       return st;
@@ -208,13 +208,13 @@ int ug_plan_create(const ug_geom* g, ug_plan** out) {
     }
     char* base = static_cast<char*>(p->d_mem);
     p->d_err = reinterpret_cast<int*>(base + a_err);
-    p->d_rope = reinterpret_cast<double*>(base + a_rope);
+    p->d_rope = reinterpret_cast<float*>(base + a_rope);
     p->d_qtiles = reinterpret_cast<QTile*>(base + a_qt);
     p->d_kvlist = reinterpret_cast<uint32_t*>(base + a_kv);
     p->d_ktiles = reinterpret_cast<KTile*>(base + a_kt);
     p->d_qlist = reinterpret_cast<uint32_t*>(base + a_ql);
     std::vector<char> host(total, 0);
-    std::memcpy(host.data() + a_rope, tables.data(), tables.size() * sizeof(double));
+    std::memcpy(host.data() + a_rope, tables.data(), tables.size() * sizeof(float));
     std::memcpy(host.data() + a_qt, p->qtiles.data(), p->qtiles.size() * sizeof(QTile));
     std::memcpy(host.data() + a_kv, p->kvlist.data(), p->kvlist.size() * sizeof(uint32_t));
     std::memcpy(host.data() + a_kt, p->ktiles.data(), p->ktiles.size() * sizeof(KTile));
@@ -437,15 +437,19 @@ int64_t ug_attn_bwd_workspace_bytes(const ug_plan* p) {
   return ((int64_t)p->g.batch * p->g.heads * (p->N + p->L) * 4 + 255) / 256 * 256;
 }
 
-int ug_hier_local_attn_bwd(const ug_plan* p, const void* q_hr, const void* k_hr,
-                           const void* v_hr, const void* q_lr, const void* k_lr,
-                           const void* v_lr, const void* o_hr, const void* o_lr,
-                           const void* do_hr, const void* do_lr, const float* lse, void* dq_hr,
-                           void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr, void* dv_lr,
-                           void* workspace, int64_t workspace_bytes, void* s) {
+}  // extern "C"
+
+namespace {
+
+int attn_bwd_checked(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
+                     const void* q_lr, const void* k_lr, const void* v_lr, const void* o_hr,
+                     const void* o_lr, const void* do_hr, const void* do_lr, const float* lse,
+                     void* dq_hr, void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr, void* dv_lr,
+                     void* workspace, int64_t workspace_bytes, bool vo_raster, void* s) {
   if (!p || !lse || !workspace) return UG_ERR_INVALID_ARG;
   if (workspace_bytes < ug_attn_bwd_workspace_bytes(p)) return UG_ERR_INVALID_ARG;
   const bool lr = p->L > 0;
+  if (!lr) q_lr = k_lr = v_lr = o_lr = do_lr = dq_lr = dk_lr = dv_lr = nullptr;
   const void* ins[10] = {q_hr, k_hr, v_hr, o_hr, do_hr, q_lr, k_lr, v_lr, o_lr, do_lr};
   void* outs[6] = {dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr};
   for (int i = 0; i < 10; ++i)
@@ -472,11 +476,38 @@ int ug_hier_local_attn_bwd(const ug_plan* p, const void* q_hr, const void* k_hr,
       if (overlap(w[i], wn[i], w[j], wn[j])) return UG_ERR_ALIAS;
   }
   if (const int st = check_device(p)) return st;
-  return launch_attention_bwd(p, q_hr, k_hr, v_hr, lr ? q_lr : nullptr, lr ? k_lr : nullptr,
-                              lr ? v_lr : nullptr, o_hr, lr ? o_lr : nullptr, do_hr,
-                              lr ? do_lr : nullptr, lse, dq_hr, dk_hr, dv_hr,
-                              lr ? dq_lr : nullptr, lr ? dk_lr : nullptr, lr ? dv_lr : nullptr,
-                              static_cast<float*>(workspace), as_stream(s));
+  return launch_attention_bwd(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr, do_lr,
+                              lse, dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr,
+                              static_cast<float*>(workspace), vo_raster, as_stream(s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int ug_hier_local_attn_bwd(const ug_plan* p, const void* q_hr, const void* k_hr,
+                           const void* v_hr, const void* q_lr, const void* k_lr,
+                           const void* v_lr, const void* o_hr, const void* o_lr,
+                           const void* do_hr, const void* do_lr, const float* lse, void* dq_hr,
+                           void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr, void* dv_lr,
+                           void* workspace, int64_t workspace_bytes, void* s) {
+  return attn_bwd_checked(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr, do_lr, lse,
+                          dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr, workspace, workspace_bytes,
+                          false, s);
+}
+
+int ug_hier_local_attn_bwd_vo_raster(const ug_plan* p, const void* q_hr, const void* k_hr,
+                                     const void* v_hr_raster, const void* q_lr,
+                                     const void* k_lr, const void* v_lr,
+                                     const void* o_hr_raster, const void* o_lr,
+                                     const void* do_hr_raster, const void* do_lr,
+                                     const float* lse, void* dq_hr, void* dk_hr,
+                                     void* dv_hr_raster, void* dq_lr, void* dk_lr, void* dv_lr,
+                                     void* workspace, int64_t workspace_bytes, void* s) {
+  if (p && !vo_raster_supported(p->g)) return UG_ERR_UNSUPPORTED;
+  return attn_bwd_checked(p, q_hr, k_hr, v_hr_raster, q_lr, k_lr, v_lr, o_hr_raster, o_lr,
+                          do_hr_raster, do_lr, lse, dq_hr, dk_hr, dv_hr_raster, dq_lr, dk_lr,
+                          dv_lr, workspace, workspace_bytes, true, s);
 }
 
 int64_t ug_layer_bwd_workspace_bytes(const ug_plan* p) {
@@ -541,21 +572,32 @@ int ug_layer_bwd(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   int st;
   if ((st = ug_permute_rope_window_first(p, q_hr, q_wf, s)) != UG_OK) return st;
   if ((st = ug_permute_rope_window_first(p, k_hr, k_wf, s)) != UG_OK) return st;
-  if ((st = ug_permute_window_first(p, v_hr, v_wf, s)) != UG_OK) return st;
-  if ((st = ug_permute_window_first(p, o_hr, o_wf, s)) != UG_OK) return st;
-  if ((st = ug_permute_window_first(p, do_hr, do_wf, s)) != UG_OK) return st;
+  // Where 128-row tiles are whole window rows, the attention backward reads
+  // v, o, dO and writes dv in raster order itself (no permutes of v, o, dO,
+  // no unpermute of dv).
+  const bool raster = vo_raster_supported(p->g);
+  if (!raster) {
+    if ((st = ug_permute_window_first(p, v_hr, v_wf, s)) != UG_OK) return st;
+    if ((st = ug_permute_window_first(p, o_hr, o_wf, s)) != UG_OK) return st;
+    if ((st = ug_permute_window_first(p, do_hr, do_wf, s)) != UG_OK) return st;
+  }
   if (lr) {
     if ((st = ug_rope_2d(p, q_lr, q_lr_r, UG_LR, s)) != UG_OK) return st;
     if ((st = ug_rope_2d(p, k_lr, k_lr_r, UG_LR, s)) != UG_OK) return st;
   }
   // global dq, dk land in the outputs in the rotated frame, then rotate back in place
-  if ((st = ug_hier_local_attn_bwd(p, q_wf, k_wf, v_wf, q_lr_r, k_lr_r, v_lr, o_wf, o_lr, do_wf,
-                                   do_lr, lse, dq_wf, dk_wf, dv_wf, dq_lr, dk_lr, dv_lr, delta,
-                                   ug_attn_bwd_workspace_bytes(p), s)) != UG_OK)
-    return st;
+  if (raster)
+    st = ug_hier_local_attn_bwd_vo_raster(p, q_wf, k_wf, v_hr, q_lr_r, k_lr_r, v_lr, o_hr, o_lr,
+                                          do_hr, do_lr, lse, dq_wf, dk_wf, dv_hr, dq_lr, dk_lr,
+                                          dv_lr, delta, ug_attn_bwd_workspace_bytes(p), s);
+  else
+    st = ug_hier_local_attn_bwd(p, q_wf, k_wf, v_wf, q_lr_r, k_lr_r, v_lr, o_wf, o_lr, do_wf,
+                                do_lr, lse, dq_wf, dk_wf, dv_wf, dq_lr, dk_lr, dv_lr, delta,
+                                ug_attn_bwd_workspace_bytes(p), s);
+  if (st != UG_OK) return st;
   if ((st = ug_unpermute_rope_bwd(p, dq_wf, dq_hr, s)) != UG_OK) return st;
   if ((st = ug_unpermute_rope_bwd(p, dk_wf, dk_hr, s)) != UG_OK) return st;
-  if ((st = ug_unpermute(p, dv_wf, dv_hr, s)) != UG_OK) return st;
+  if (!raster && (st = ug_unpermute(p, dv_wf, dv_hr, s)) != UG_OK) return st;
   if (lr) {
     if ((st = ug_rope_2d_bwd(p, dq_lr, dq_lr, UG_LR, s)) != UG_OK) return st;
     if ((st = ug_rope_2d_bwd(p, dk_lr, dk_lr, UG_LR, s)) != UG_OK) return st;

@@ -46,6 +46,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "ug_debug.h"
 #include "ug_internal.h"
 #include "ug_per_device.h"
 #include "ug_tc.cuh"
@@ -86,6 +87,7 @@ struct AttnParams {
   // tile = 128 / win_w whole rows of one window) and raster-order o_hr.
   int32_t vo_raster;
   int32_t grid_w, win_h, win_w;
+  int32_t kv_len;  // entries in kvlist (debug-build range checks)
 };
 
 // Raster index of the high-res token at window-first position p.
@@ -160,6 +162,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain, 1);
     // A CTA that starts after another one gave up does no work.
     *abort = *reinterpret_cast<volatile int*>(err) != 0 ? 1u : 0u;
+#if UG_DEBUG
+    // the CTA's slice of the block list, and every block in it, in range
+    bool lst = qt.list_off >= 0 && qt.list_len >= 1 && qt.list_off + qt.list_len <= P.kv_len;
+    for (int j = 0; lst && j < nblk; ++j) {
+      const uint32_t e = P.kvlist[qt.list_off + j];
+      const int n = (e & kBlockLowres) ? P.L : P.N;
+      lst = (int64_t)(e & kBlockIndexMask) * kKeysPerBlock < n;
+    }
+    const int ntq = qt.lowres ? P.L : P.N;
+    if (!dbg_ok(lst && qt.q0 >= 0 && qt.q0 < ntq, err)) *abort = 1u;
+#endif
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kMmaWarp) {
@@ -404,9 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       fence_after();
       const int ntok = qt.lowres ? P.L : P.N;
-      const bool valid = tok < ntok;
+      bool valid = tok < ntok;
       const float inv_l = 1.0f / l;
       const int orow = (!qt.lowres && P.vo_raster && valid) ? raster_of(tok, P) : tok;
+      if (valid) valid = dbg_ok(orow >= 0 && orow < ntok, err);
       __nv_bfloat16* dst = (qt.lowres ? P.o_lr : P.o_hr) +
                            (((int64_t)b * ntok + orow) * P.heads + head) * D;
 #pragma unroll 1
@@ -477,6 +491,7 @@ int launch_d(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v
   P.grid_w = p->g.grid_w;
   P.win_h = p->g.win_h;
   P.win_w = p->g.win_w;
+  P.kv_len = (int32_t)p->kvlist.size();
   if (const int pst = prepare_attention(p->device)) return pst;
   const dim3 grid((unsigned)p->qtiles.size(), (unsigned)H, (unsigned)B);
   hier_attn_kernel<D><<<grid, kThreads, Layout<D>::kAlloc, st>>>(m[0], m[1], m[2], m[3], m[4],

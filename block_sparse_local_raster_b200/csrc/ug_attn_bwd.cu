@@ -34,6 +34,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "ug_debug.h"
 #include "ug_internal.h"
 #include "ug_per_device.h"
 #include "ug_tc.cuh"
@@ -64,21 +65,70 @@ struct BwdParams {
   int32_t N, L, T, nwx, radius, heads;
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)
+  int32_t kv_len, q_len;  // entries in kvlist / qlist (debug-build range checks)
+  // Raster-order high-res V, O, dO and dV (V and dO read through 5-D tensor
+  // maps, one 128-row tile = 128 / win_w whole rows of one window; dV rows
+  // scattered to their raster positions).
+  int32_t vo_raster;
+  int32_t grid_w, win_h, win_w;
 };
+
+// Raster index of the high-res token at window-first position p.
+__device__ __forceinline__ int raster_of(int p, int T, int nwx, int win_h, int win_w,
+                                         int grid_w) {
+  const int w = p / T, l = p - (p / T) * T;
+  const int wy = w / nwx, wx = w - (w / nwx) * nwx;
+  const int ly = l / win_w, lx = l - (l / win_w) * win_w;
+  return (wy * win_h + ly) * grid_w + wx * win_w + lx;
+}
+
+// One 128-row tile (rows row0.. of the window-first order, one head) of a
+// high-res tensor into shared memory: through the 4-D map of a window-first
+// tensor, or the 5-D map of a raster one (the tile is 128 / win_w whole rows
+// of one window, landing in window-first order).
+template <int kRegions>
+__device__ __forceinline__ void load_hr_tile(uint32_t dst, const CUtensorMap* map, bool raster,
+                                             int row0, int head, int b, const BwdParams& P,
+                                             uint32_t bar) {
+  if (raster) {
+    const int w = row0 / P.T, ly0 = (row0 - (row0 / P.T) * P.T) / P.win_w;
+    const int wy = w / P.nwx, wx = w - (w / P.nwx) * P.nwx;
+    for (int r = 0; r < kRegions; ++r)
+      tma_load_5d(dst + r * kRowsPerTile * 128, map, r * 64, head, wx * P.win_w,
+                  wy * P.win_h + ly0, b, bar);
+  } else {
+    for (int r = 0; r < kRegions; ++r)
+      tma_load_4d(dst + r * kRowsPerTile * 128, map, r * 64, head, row0, b, bar);
+  }
+}
+
+// Debug build: a list slice [off, off + len) inside a list of n entries, and
+// every 128-row block it names inside its token set.
+__device__ __forceinline__ bool list_in_range(const uint32_t* list, int off, int len, int n,
+                                              int n_hr, int n_lr) {
+  bool ok = off >= 0 && len >= 0 && off + len <= n;
+  for (int j = 0; ok && j < len; ++j) {
+    const uint32_t e = list[off + j];
+    ok = (int64_t)(e & kBlockIndexMask) * kRowsPerTile < ((e & kBlockLowres) ? n_lr : n_hr);
+  }
+  return ok;
+}
 
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ delta
 
 // D[b, h, r] = sum_c dO[b, r, h, c] * O[b, r, h, c] (fp32), for the high-res
-// rows then the global rows.  One warp per token row; D/8 lanes per head.
+// rows (window-first order r; O and dO window-first, or raster with
+// `raster`) then the global rows.  One warp per token row; D/8 lanes per head.
 template <int D>
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o_hr,
                                                     const __nv_bfloat16* __restrict__ do_hr,
                                                     const __nv_bfloat16* __restrict__ o_lr,
                                                     const __nv_bfloat16* __restrict__ do_lr,
                                                     float* __restrict__ delta, int B, int N,
-                                                    int L, int H) {
+                                                    int L, int H, int raster, int T, int nwx,
+                                                    int win_h, int win_w, int grid_w) {
   constexpr int kCh = D / 8;        // 16-byte chunks per head
   constexpr int kHeadsPer = 32 / kCh;
   const int lane = threadIdx.x & 31;
@@ -91,7 +141,9 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
     const bool lr = tok >= N;
     const int t = lr ? tok - N : tok;
     const int n = lr ? L : N;
-    const int64_t base = ((int64_t)b * n + t) * H * D;
+    // with raster o_hr / do_hr, window-first row t sits at its raster position
+    const int mt = (!lr && raster) ? raster_of(t, T, nwx, win_h, win_w, grid_w) : t;
+    const int64_t base = ((int64_t)b * n + mt) * H * D;
     const uint4* o = reinterpret_cast<const uint4*>((lr ? o_lr : o_hr) + base);
     const uint4* g = reinterpret_cast<const uint4*>((lr ? do_lr : do_hr) + base);
     for (int h0 = 0; h0 < H; h0 += kHeadsPer) {
@@ -276,6 +328,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(dq_done, 1);
     mbar_init(drain, 1);
     *abort = *reinterpret_cast<volatile int*>(err) != 0 ? 1u : 0u;
+#if UG_DEBUG
+    if (!dbg_ok(list_in_range(P.kvlist, qt.list_off, nblk, P.kv_len, P.N, P.L) && qt.q0 >= 0 &&
+                    qt.q0 < (qt.lowres ? P.L : P.N),
+                err))
+      *abort = 1u;
+#endif
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kBwdMma) {
@@ -307,12 +365,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdProducer) {
     if (lane == 0) {
       mbar_expect_tx(q_full, 2 * kTile);
-      for (int r = 0; r < kRegions; ++r) {
+      for (int r = 0; r < kRegions; ++r)
         tma_load_4d(sbase + Lay::kQ + r * kRowsPerTile * 128, qt.lowres ? &tm_q_lr : &tm_q_hr,
                     r * 64, head, q0, b, q_full);
-        tma_load_4d(sbase + Lay::kDO + r * kRowsPerTile * 128,
-                    qt.lowres ? &tm_do_lr : &tm_do_hr, r * 64, head, q0, b, q_full);
-      }
+      load_hr_tile<kRegions>(sbase + Lay::kDO, qt.lowres ? &tm_do_lr : &tm_do_hr,
+                             !qt.lowres && P.vo_raster, q0, head, b, P, q_full);
       int it = 0;
       bool ok = true;
       for (int j = 0; j < nblk && ok; ++j) {
@@ -326,9 +383,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             break;
           }
           mbar_expect_tx(kv_full(slot(it)), kTile);
-          for (int r = 0; r < kRegions; ++r)
-            tma_load_4d(sbase + Lay::kKV + slot(it) * kTile + r * kKeysPerBlock * 128, m, r * 64,
-                        head, k0, b, kv_full(slot(it)));
+          load_hr_tile<kRegions>(sbase + Lay::kKV + slot(it) * kTile, m,
+                                 kv == 1 && !lr && P.vo_raster, k0, head, b, P,
+                                 kv_full(slot(it)));
         }
       }
       for (int i = (it > kRing ? it - kRing : 0); i < it; ++i) drain_wait(kv_full(slot(i)), phase(i));
@@ -583,6 +640,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(group(0), kRowsPerTile);
     mbar_init(group(1), kRowsPerTile);
     *abort = *reinterpret_cast<volatile int*>(err) != 0 ? 1u : 0u;
+#if UG_DEBUG
+    if (!dbg_ok(list_in_range(P.qlist, kt.list_off, nq, P.q_len, P.N, P.L) && kt.k0 >= 0 &&
+                    kt.k0 < nk,
+                err))
+      *abort = 1u;
+#endif
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kBwdMma) {
@@ -614,12 +677,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdProducer) {
     if (lane == 0) {
       mbar_expect_tx(kv_full, 2 * kTile);
-      for (int r = 0; r < kRegions; ++r) {
+      for (int r = 0; r < kRegions; ++r)
         tma_load_4d(sbase + Lay::kK + r * kKeysPerBlock * 128, kt.lowres ? &tm_k_lr : &tm_k_hr,
                     r * 64, head, kt.k0, b, kv_full);
-        tma_load_4d(sbase + Lay::kV + r * kKeysPerBlock * 128, kt.lowres ? &tm_v_lr : &tm_v_hr,
-                    r * 64, head, kt.k0, b, kv_full);
-      }
+      load_hr_tile<kRegions>(sbase + Lay::kV, kt.lowres ? &tm_v_lr : &tm_v_hr,
+                             !kt.lowres && P.vo_raster, kt.k0, head, b, P, kv_full);
       int it = 0;
       bool ok = true;
       for (int i = 0; i < nq && ok; ++i) {
@@ -633,9 +695,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             break;
           }
           mbar_expect_tx(ring_full(slot(it)), kTile);
-          for (int r = 0; r < kRegions; ++r)
-            tma_load_4d(sbase + Lay::kRingOff + slot(it) * kTile + r * kRowsPerTile * 128, m,
-                        r * 64, head, q0, b, ring_full(slot(it)));
+          load_hr_tile<kRegions>(sbase + Lay::kRingOff + slot(it) * kTile, m,
+                                 x == 1 && !lr && P.vo_raster, q0, head, b, P,
+                                 ring_full(slot(it)));
         }
       }
       for (int i = (it > kRing ? it - kRing : 0); i < it; ++i)
@@ -781,9 +843,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) {
       fence_after();
       // warpgroup 0 writes dV, warpgroup 1 writes dK (scaled)
-      const bool valid = key < nk;
+      bool valid = key < nk;
+      // dV of high-res keys goes to its raster row when dV is raster-ordered
+      const int orow = (valid && g == 0 && !kt.lowres && P.vo_raster)
+                           ? raster_of(key, P.T, P.nwx, P.win_h, P.win_w, P.grid_w)
+                           : key;
+      if (valid) valid = dbg_ok(orow >= 0 && orow < nk, err);
       __nv_bfloat16* dst = (g == 0 ? (kt.lowres ? P.dv_lr : P.dv_hr) : (kt.lowres ? P.dk_lr : P.dk_hr)) +
-                           (((int64_t)b * nk + key) * P.heads + head) * D;
+                           (((int64_t)b * nk + orow) * P.heads + head) * D;
       const float k = g == 0 ? 1.0f : P.scale;
       const uint32_t tacc = tmem + lane_base + (g == 0 ? 256u : 384u);
 #pragma unroll 1
@@ -822,7 +889,7 @@ int launch_bwd_d(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
                  const void* q_lr, const void* k_lr, const void* v_lr, const void* o_hr,
                  const void* o_lr, const void* do_hr, const void* do_lr, const float* lse,
                  void* dq_hr, void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr, void* dv_lr,
-                 float* delta, cudaStream_t st) {
+                 float* delta, bool vo_raster, cudaStream_t st) {
   const int64_t B = p->g.batch;
   const int H = p->g.heads;
   const bool has_lr = p->L > 0;
@@ -831,9 +898,13 @@ int launch_bwd_d(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   const void* hr[4] = {q_hr, k_hr, v_hr, do_hr};
   const void* lr[4] = {has_lr ? q_lr : q_hr, has_lr ? k_lr : k_hr, has_lr ? v_lr : v_hr,
                        has_lr ? do_lr : do_hr};
-  for (int i = 0; i < 4; ++i)
-    if (!make_map(&m[i], hr[i], B, p->N, H, D) || !make_map(&m[4 + i], lr[i], B, nl, H, D))
-      return UG_ERR_CUDA;
+  for (int i = 0; i < 4; ++i) {
+    const bool ok_hr = (vo_raster && i >= 2)
+                           ? make_map_raster(&m[i], hr[i], B, p->g.grid_h, p->g.grid_w, H, D,
+                                             p->g.win_w)
+                           : make_map(&m[i], hr[i], B, p->N, H, D);
+    if (!ok_hr || !make_map(&m[4 + i], lr[i], B, nl, H, D)) return UG_ERR_CUDA;
+  }
   BwdParams P;
   P.qtiles = p->d_qtiles;
   P.kvlist = p->d_kvlist;
@@ -857,6 +928,12 @@ int launch_bwd_d(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
   P.heads = H;
   P.scale = p->scale;
   P.scale_log2 = p->scale * kLog2e;
+  P.kv_len = (int32_t)p->kvlist.size();
+  P.q_len = (int32_t)p->qlist.size();
+  P.vo_raster = vo_raster ? 1 : 0;
+  P.grid_w = p->g.grid_w;
+  P.win_h = p->g.win_h;
+  P.win_w = p->g.win_w;
   if (const int pst = prepare_attention_bwd(p->device)) return pst;
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device);
@@ -866,7 +943,7 @@ int launch_bwd_d(const ug_plan* p, const void* q_hr, const void* k_hr, const voi
       static_cast<const __nv_bfloat16*>(o_hr), static_cast<const __nv_bfloat16*>(do_hr),
       static_cast<const __nv_bfloat16*>(has_lr ? o_lr : o_hr),
       static_cast<const __nv_bfloat16*>(has_lr ? do_lr : do_hr), delta, (int)B, (int)p->N,
-      (int)p->L, H);
+      (int)p->L, H, vo_raster ? 1 : 0, (int)p->T, p->nwx, p->g.win_h, p->g.win_w, p->g.grid_w);
   const dim3 gq((unsigned)(2 * p->qtiles.size()), (unsigned)H, (unsigned)B);
   dq_kernel<D><<<gq, kBwdThreads, DqLayout<D>::kAlloc, st>>>(m[0], m[1], m[2], m[3], m[4], m[5],
                                                              m[6], m[7], P);
@@ -902,13 +979,13 @@ int launch_attention_bwd(const ug_plan* p, const void* q_hr, const void* k_hr, c
                          const void* q_lr, const void* k_lr, const void* v_lr, const void* o_hr,
                          const void* o_lr, const void* do_hr, const void* do_lr, const float* lse,
                          void* dq_hr, void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr,
-                         void* dv_lr, float* delta, cudaStream_t st) {
+                         void* dv_lr, float* delta, bool vo_raster, cudaStream_t st) {
   if (p->g.head_dim == 128)
     return launch_bwd_d<128>(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr, do_lr, lse,
-                             dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr, delta, st);
+                             dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr, delta, vo_raster, st);
   if (p->g.head_dim == 64)
     return launch_bwd_d<64>(p, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr, do_lr, lse,
-                            dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr, delta, st);
+                            dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr, delta, vo_raster, st);
   return UG_ERR_UNSUPPORTED;
 }
 

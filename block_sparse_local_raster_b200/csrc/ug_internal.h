@@ -45,13 +45,16 @@ constexpr uint32_t kBlockIndexMask = (1u << 29) - 1;
 constexpr uint32_t kBlockLowres = 1u << 29;
 constexpr uint32_t kBlockMasked = 1u << 30;
 
-// Offsets (in elements) of the RoPE tables inside the plan's table buffer.
-// Each table is [coordinate][pair k]; cos and sin separately.  The values
-// are the fp32-rounded cos/sin, held in fp64 (exactly) so that the kernels
-// need no conversion to form exact fp64 products.
+// Offsets (in elements) of the RoPE tables inside the plan's table buffer,
+// for one axis of one token set.  Each table is [coordinate][pair k]; the
+// fp32-rounded cos and sin are each stored split, c = hi + lo with hi the
+// leading 16 bits of c's significand (ug_rope_math.h), every table and row
+// 16-byte aligned.
+struct AxisTables {
+  int64_t cos_hi, sin_hi, cos_lo, sin_lo;
+};
 struct RopeTables {
-  int64_t hr_y_cos, hr_y_sin, hr_x_cos, hr_x_sin;
-  int64_t lr_y_cos, lr_y_sin, lr_x_cos, lr_x_sin;
+  AxisTables hr_y, hr_x, lr_y, lr_x;
   int64_t total;
 };
 
@@ -81,7 +84,7 @@ struct ug_plan {
   ug::RopeTables rope;
 
   void* d_mem;             // one device allocation holding everything below
-  double* d_rope;          // RoPE tables
+  float* d_rope;           // RoPE tables
   ug::QTile* d_qtiles;     // attention query CTAs
   uint32_t* d_kvlist;      // attention key-block lists
   ug::KTile* d_ktiles;     // backward key CTAs
@@ -114,17 +117,19 @@ int launch_attention_bwd(const ug_plan* p, const void* q_hr, const void* k_hr, c
                          const void* q_lr, const void* k_lr, const void* v_lr, const void* o_hr,
                          const void* o_lr, const void* do_hr, const void* do_lr, const float* lse,
                          void* dq_hr, void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr,
-                         void* dv_lr, float* delta, cudaStream_t s);
+                         void* dv_lr, float* delta, bool vo_raster, cudaStream_t s);
 int launch_warm_start(const ug_warm_start_params* p, const float* x_lr, const float* noise,
                       float* out, cudaStream_t s);
 int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                      const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
                      void* o_lr, float* lse, bool vo_raster, cudaStream_t s);
 // Per-device set-up, done once per device and run by ug_plan_create with the
-// plan's device current: the attention kernels' shared-memory opt-in, and the
-// device address of the static scratch of ug_layer_fwd_static_scratch.
+// plan's device current: the attention and RoPE kernels' shared-memory
+// opt-in, and the device address of the static scratch of
+// ug_layer_fwd_static_scratch.
 int prepare_attention(int device);
 int prepare_attention_bwd(int device);
+int prepare_rope(int device);
 int prepare_static_scratch(int device);
 // Whether a 128-key tile is always 128 / win_w whole rows of one window, so
 // that raster-order V can be read tile by tile.

@@ -9,6 +9,7 @@
 // once per segment.  HBM-bound: 2 bytes moved per byte of tensor.
 #include <cstdint>
 
+#include "ug_debug.h"
 #include "ug_internal.h"
 
 namespace ug {
@@ -26,6 +27,8 @@ struct PermuteArgs {
   int32_t seg_chunks;  // win_w * row_chunks
   int32_t grid_h, grid_w, win_h, win_w, nwx, T;
   int32_t inverse;     // 0: raster -> window-first, 1: window-first -> raster
+  int64_t batch;       // B (debug-build range checks)
+  int* err;            // the plan's error word
 };
 
 __global__ void __launch_bounds__(kThreads) permute_kernel(const PermuteArgs a) {
@@ -39,6 +42,11 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const PermuteArgs a) 
     const int64_t p0 = ((int64_t)wy * a.nwx + wx) * a.T + (int64_t)ly * a.win_w;  // window-first
     const int64_t s_tok = a.inverse ? p0 : r0;
     const int64_t d_tok = a.inverse ? r0 : p0;
+    // both runs of win_w tokens lie inside their batch element's tensor
+    if (!dbg_ok(b < a.batch && s_tok >= 0 && d_tok >= 0 && s_tok + a.win_w <= a.n_tok &&
+                    d_tok + a.win_w <= a.n_tok,
+                a.err))
+      continue;
     const uint4* __restrict__ s = a.src + (b * a.n_tok + s_tok) * a.row_chunks;
     uint4* __restrict__ d = a.dst + (b * a.n_tok + d_tok) * a.row_chunks;
     int32_t c = threadIdx.x;
@@ -70,6 +78,8 @@ int launch_permute(const ug_plan* p, const void* src, void* dst, bool inverse, c
   a.seg_chunks = a.win_w * a.row_chunks;
   a.n_seg = (int64_t)p->g.batch * p->g.grid_h * p->nwx;
   a.inverse = inverse ? 1 : 0;
+  a.batch = p->g.batch;
+  a.err = p->d_err;
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device);
   const int64_t blocks = std::min<int64_t>(a.n_seg, (int64_t)sms * (2048 / kThreads));

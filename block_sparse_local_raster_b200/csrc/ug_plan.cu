@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "ug_internal.h"
+#include "ug_rope_math.h"
 
 namespace ug {
 
@@ -177,15 +178,24 @@ void build_backward_lists(const ug_geom& g, const std::vector<int32_t>& nbr_off,
 
 // f_k = theta^(-2k/a) (one pow in fp64); angle = position * f_k (one fp64
 // product); cos and sin from the C library in fp64, rounded to fp32.
-static void axis_table(const std::vector<double>& pos, int a, double theta, float* c, float* s) {
+// cos and sin of pos * theta^(-2k/a) for every position and pair k: the
+// angle in fp64, cos/sin from the C library, rounded to fp32 once, then
+// stored split into the fp32 high part (leading 16 significand bits) and the
+// remainder, which add back to the fp32 value exactly.
+static void axis_table(const std::vector<double>& pos, int a, double theta, float* out,
+                       const AxisTables& t) {
   const int m = a / 2;
   std::vector<double> f((size_t)m);
   for (int k = 0; k < m; ++k) f[(size_t)k] = std::pow(theta, -2.0 * k / a);
   for (size_t i = 0; i < pos.size(); ++i)
     for (int k = 0; k < m; ++k) {
       const double ang = pos[i] * f[(size_t)k];
-      c[i * m + k] = (float)std::cos(ang);
-      s[i * m + k] = (float)std::sin(ang);
+      const float c = (float)std::cos(ang), s = (float)std::sin(ang);
+      const size_t at = i * m + k;
+      out[t.cos_hi + at] = rope_math::split_hi(c);
+      out[t.cos_lo + at] = rope_math::split_lo(c);
+      out[t.sin_hi + at] = rope_math::split_hi(s);
+      out[t.sin_lo + at] = rope_math::split_lo(s);
     }
 }
 
@@ -197,14 +207,18 @@ void build_rope_tables(const ug_geom& g, RopeTables& o, std::vector<float>& data
     at += (n + 3) / 4 * 4;  // keep every table 16-byte aligned
     return r;
   };
-  o.hr_y_cos = take(g.grid_h * my);
-  o.hr_y_sin = take(g.grid_h * my);
-  o.hr_x_cos = take(g.grid_w * mx);
-  o.hr_x_sin = take(g.grid_w * mx);
-  o.lr_y_cos = take(g.lr_h * my);
-  o.lr_y_sin = take(g.lr_h * my);
-  o.lr_x_cos = take(g.lr_w * mx);
-  o.lr_x_sin = take(g.lr_w * mx);
+  auto axis = [&](int64_t n) {
+    AxisTables t;
+    t.cos_hi = take(n);
+    t.sin_hi = take(n);
+    t.cos_lo = take(n);
+    t.sin_lo = take(n);
+    return t;
+  };
+  o.hr_y = axis(g.grid_h * my);
+  o.hr_x = axis(g.grid_w * mx);
+  o.lr_y = axis(g.lr_h * my);
+  o.lr_x = axis(g.lr_w * mx);
   o.total = std::max<int64_t>(at, 4);
   data.assign((size_t)o.total, 0.0f);
   std::vector<double> py, px, ly, lx;
@@ -212,11 +226,11 @@ void build_rope_tables(const ug_geom& g, RopeTables& o, std::vector<float>& data
   for (int i = 0; i < g.grid_w; ++i) px.push_back((double)i);
   for (int i = 0; i < g.lr_h; ++i) ly.push_back(g.rho * (double)i);
   for (int i = 0; i < g.lr_w; ++i) lx.push_back(g.rho * (double)i);
-  axis_table(py, g.rope_dim_y, g.rope_theta, &data[(size_t)o.hr_y_cos], &data[(size_t)o.hr_y_sin]);
-  axis_table(px, g.rope_dim_x, g.rope_theta, &data[(size_t)o.hr_x_cos], &data[(size_t)o.hr_x_sin]);
+  axis_table(py, g.rope_dim_y, g.rope_theta, data.data(), o.hr_y);
+  axis_table(px, g.rope_dim_x, g.rope_theta, data.data(), o.hr_x);
   if (g.lr_h > 0) {
-    axis_table(ly, g.rope_dim_y, g.rope_theta, &data[(size_t)o.lr_y_cos], &data[(size_t)o.lr_y_sin]);
-    axis_table(lx, g.rope_dim_x, g.rope_theta, &data[(size_t)o.lr_x_cos], &data[(size_t)o.lr_x_sin]);
+    axis_table(ly, g.rope_dim_y, g.rope_theta, data.data(), o.lr_y);
+    axis_table(lx, g.rope_dim_x, g.rope_theta, data.data(), o.lr_x);
   }
 }
 

@@ -16,6 +16,9 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libug.so")
+# The same library built with -DUG_DEBUG=1: a range check before every global
+# access whose index a kernel computes (failures reach ug_check_error).
+LIB_DEBUG_PATH = os.path.join(_HERE, "libug_debug.so")
 
 UG_OK = 0
 UG_ERR_INVALID_ARG = 1
@@ -40,7 +43,8 @@ EXPORTS = (
     "ug_layer_workspace_bytes", "ug_layer_fwd", "ug_layer_fwd_static_scratch",
     "ug_plan_set_wait_timeout", "ug_check_error", "ug_warm_start",
     "ug_rope_2d_bwd", "ug_unpermute_rope_bwd", "ug_attn_bwd_workspace_bytes",
-    "ug_hier_local_attn_bwd", "ug_layer_bwd_workspace_bytes", "ug_layer_bwd",
+    "ug_hier_local_attn_bwd", "ug_hier_local_attn_bwd_vo_raster",
+    "ug_layer_bwd_workspace_bytes", "ug_layer_bwd",
 )
 
 # Capacity of the static scratch of ug_layer_fwd_static_scratch (ug.h).
@@ -74,17 +78,41 @@ class ug_warm_start_params(ctypes.Structure):
 
 
 _lib = None
+_loaded = {}
 
 
 def lib() -> ctypes.CDLL:
-    """Load libug.so once (raises if it was not built)."""
+    """The library the binding currently uses (LIB_PATH unless use_library
+    chose another); loaded once per path, raises if it was not built."""
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+    _lib = _load(LIB_PATH)
+    return _lib
+
+
+def use_library(path: str) -> ctypes.CDLL:
+    """Makes the library at path (e.g. LIB_DEBUG_PATH) the one that new plans
+    and module-level calls use; plans already created keep theirs.  Returns
+    the library that was in use before."""
+    global _lib
+    prev = lib()
+    _lib = _load(path)
+    return prev
+
+
+def _set_library(L: ctypes.CDLL) -> None:
+    global _lib
+    _lib = L
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if path in _loaded:
+        return _loaded[path]
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
                            "`python -m block_sparse_local_raster_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     P, I32, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
     G = ctypes.POINTER(ug_geom)
     pi32 = ctypes.POINTER(ctypes.c_int32)
@@ -117,6 +145,7 @@ def lib() -> ctypes.CDLL:
         "ug_unpermute_rope_bwd": (I32, [P, P, P, P]),
         "ug_attn_bwd_workspace_bytes": (I64, [P]),
         "ug_hier_local_attn_bwd": (I32, [P] + [P] * 17 + [P, I64, P]),
+        "ug_hier_local_attn_bwd_vo_raster": (I32, [P] + [P] * 17 + [P, I64, P]),
         "ug_layer_bwd_workspace_bytes": (I64, [P]),
         "ug_layer_bwd": (I32, [P] + [P] * 17 + [P, I64, P]),
     }
@@ -124,7 +153,7 @@ def lib() -> ctypes.CDLL:
         f = getattr(L, name)
         f.restype = res
         f.argtypes = args
-    _lib = L
+    _loaded[path] = L
     return L
 
 
@@ -205,18 +234,19 @@ class Plan:
         self.geom_kw = dict(geom)
         self.g = make_geom(**geom)
         h = ctypes.c_void_p()
-        _check(lib().ug_plan_create(ctypes.byref(self.g), ctypes.byref(h)), "ug_plan_create")
+        self._L = lib()  # a plan is valid only in the library that created it
+        _check(self._L.ug_plan_create(ctypes.byref(self.g), ctypes.byref(h)), "ug_plan_create")
         self.handle = h
 
     def close(self):
         if self.handle:
-            _check(lib().ug_plan_destroy(self.handle), "ug_plan_destroy")
+            _check(self._L.ug_plan_destroy(self.handle), "ug_plan_destroy")
             self.handle = None
 
     def __del__(self):
         try:
             if getattr(self, "handle", None):
-                lib().ug_plan_destroy(self.handle)
+                self._L.ug_plan_destroy(self.handle)
                 self.handle = None
         except Exception:
             pass
@@ -224,45 +254,45 @@ class Plan:
     # -- host-side views ---------------------------------------------------
     def index_maps(self):
         n = [ctypes.c_int64() for _ in range(3)]
-        _check(lib().ug_index_map_sizes(ctypes.byref(self.g), *[ctypes.byref(x) for x in n]),
+        _check(self._L.ug_index_map_sizes(ctypes.byref(self.g), *[ctypes.byref(x) for x in n]),
                "ug_index_map_sizes")
         arrs = [np.zeros(x.value, dtype=np.int32) for x in n]
         ptrs = [a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) for a in arrs]
-        _check(lib().ug_get_index_maps(self.handle, *ptrs), "ug_get_index_maps")
+        _check(self._L.ug_get_index_maps(self.handle, *ptrs), "ug_get_index_maps")
         return tuple(arrs)
 
     def workspace_bytes(self) -> int:
-        return int(lib().ug_layer_workspace_bytes(self.handle))
+        return int(self._L.ug_layer_workspace_bytes(self.handle))
 
     # -- the four steps --------------------------------------------------------
     def permute_window_first(self, src, dst, stream=None) -> int:
-        return lib().ug_permute_window_first(self.handle, _ptr(src), _ptr(dst), _stream(stream))
+        return self._L.ug_permute_window_first(self.handle, _ptr(src), _ptr(dst), _stream(stream))
 
     def permute_rope_window_first(self, src, dst, stream=None) -> int:
-        return lib().ug_permute_rope_window_first(self.handle, _ptr(src), _ptr(dst),
+        return self._L.ug_permute_rope_window_first(self.handle, _ptr(src), _ptr(dst),
                                                   _stream(stream))
 
     def unpermute(self, src, dst, stream=None) -> int:
-        return lib().ug_unpermute(self.handle, _ptr(src), _ptr(dst), _stream(stream))
+        return self._L.ug_unpermute(self.handle, _ptr(src), _ptr(dst), _stream(stream))
 
     def rope_2d(self, x, y, token_set: int, stream=None) -> int:
-        return lib().ug_rope_2d(self.handle, _ptr(x), _ptr(y), int(token_set), _stream(stream))
+        return self._L.ug_rope_2d(self.handle, _ptr(x), _ptr(y), int(token_set), _stream(stream))
 
     def hier_local_attn_fwd(self, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse=None,
                             stream=None) -> int:
-        return lib().ug_hier_local_attn_fwd(
+        return self._L.ug_hier_local_attn_fwd(
             self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr), _ptr(q_lr), _ptr(k_lr), _ptr(v_lr),
             _ptr(o_hr), _ptr(o_lr), _ptr(lse), _stream(stream))
 
     def hier_local_attn_fwd_vo_raster(self, q_hr, k_hr, v_hr_raster, q_lr, k_lr, v_lr,
                                       o_hr_raster, o_lr, lse=None, stream=None) -> int:
-        return lib().ug_hier_local_attn_fwd_vo_raster(
+        return self._L.ug_hier_local_attn_fwd_vo_raster(
             self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr_raster), _ptr(q_lr), _ptr(k_lr),
             _ptr(v_lr), _ptr(o_hr_raster), _ptr(o_lr), _ptr(lse), _stream(stream))
 
     def layer_fwd(self, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, workspace,
                   stream=None) -> int:
-        return lib().ug_layer_fwd(
+        return self._L.ug_layer_fwd(
             self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr), _ptr(q_lr), _ptr(k_lr), _ptr(v_lr),
             _ptr(o_hr), _ptr(o_lr), _ptr(lse), _ptr(workspace),
             ctypes.c_int64(workspace.numel() * workspace.element_size()), _stream(stream))
@@ -271,37 +301,47 @@ class Plan:
                                  stream=None) -> int:
         """The layer without a caller workspace: its intermediates live in the
         library's static device scratch (no device allocation on this call)."""
-        return lib().ug_layer_fwd_static_scratch(
+        return self._L.ug_layer_fwd_static_scratch(
             self.handle, _ptr(q_hr), _ptr(k_hr), _ptr(v_hr), _ptr(q_lr), _ptr(k_lr), _ptr(v_lr),
             _ptr(o_hr), _ptr(o_lr), _ptr(lse), _stream(stream))
 
     def set_wait_timeout(self, ns: int) -> int:
-        return lib().ug_plan_set_wait_timeout(self.handle, ctypes.c_int64(int(ns)))
+        return self._L.ug_plan_set_wait_timeout(self.handle, ctypes.c_int64(int(ns)))
 
     def check_error(self, stream=None) -> int:
-        return lib().ug_check_error(self.handle, _stream(stream))
+        return self._L.ug_check_error(self.handle, _stream(stream))
 
     # -- backward ----------------------------------------------------------------
     def rope_2d_bwd(self, dy, dx, token_set: int, stream=None) -> int:
-        return lib().ug_rope_2d_bwd(self.handle, _ptr(dy), _ptr(dx), int(token_set),
+        return self._L.ug_rope_2d_bwd(self.handle, _ptr(dy), _ptr(dx), int(token_set),
                                     _stream(stream))
 
     def unpermute_rope_bwd(self, src_wf, dst_raster, stream=None) -> int:
-        return lib().ug_unpermute_rope_bwd(self.handle, _ptr(src_wf), _ptr(dst_raster),
+        return self._L.ug_unpermute_rope_bwd(self.handle, _ptr(src_wf), _ptr(dst_raster),
                                            _stream(stream))
 
     def attn_bwd_workspace_bytes(self) -> int:
-        return int(lib().ug_attn_bwd_workspace_bytes(self.handle))
+        return int(self._L.ug_attn_bwd_workspace_bytes(self.handle))
 
     def layer_bwd_workspace_bytes(self) -> int:
-        return int(lib().ug_layer_bwd_workspace_bytes(self.handle))
+        return int(self._L.ug_layer_bwd_workspace_bytes(self.handle))
 
     def hier_local_attn_bwd(self, q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr, do_lr,
                             lse, dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr, workspace,
                             stream=None) -> int:
         args = (q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, do_hr, do_lr, lse, dq_hr, dk_hr,
                 dv_hr, dq_lr, dk_lr, dv_lr, workspace)
-        return lib().ug_hier_local_attn_bwd(
+        return self._L.ug_hier_local_attn_bwd(
+            self.handle, *[_ptr(a) for a in args],
+            ctypes.c_int64(workspace.numel() * workspace.element_size()), _stream(stream))
+
+    def hier_local_attn_bwd_vo_raster(self, q_hr, k_hr, v_hr_raster, q_lr, k_lr, v_lr,
+                                      o_hr_raster, o_lr, do_hr_raster, do_lr, lse, dq_hr, dk_hr,
+                                      dv_hr_raster, dq_lr, dk_lr, dv_lr, workspace,
+                                      stream=None) -> int:
+        args = (q_hr, k_hr, v_hr_raster, q_lr, k_lr, v_lr, o_hr_raster, o_lr, do_hr_raster,
+                do_lr, lse, dq_hr, dk_hr, dv_hr_raster, dq_lr, dk_lr, dv_lr, workspace)
+        return self._L.ug_hier_local_attn_bwd_vo_raster(
             self.handle, *[_ptr(a) for a in args],
             ctypes.c_int64(workspace.numel() * workspace.element_size()), _stream(stream))
 
@@ -309,7 +349,7 @@ class Plan:
                   dq_hr, dk_hr, dv_hr, dq_lr, dk_lr, dv_lr, workspace, stream=None) -> int:
         args = (q_hr, k_hr, v_hr, q_lr, k_lr, v_lr, o_hr, o_lr, lse, do_hr, do_lr, dq_hr, dk_hr,
                 dv_hr, dq_lr, dk_lr, dv_lr, workspace)
-        return lib().ug_layer_bwd(
+        return self._L.ug_layer_bwd(
             self.handle, *[_ptr(a) for a in args],
             ctypes.c_int64(workspace.numel() * workspace.element_size()), _stream(stream))
 

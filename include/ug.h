@@ -329,6 +329,23 @@ int ug_hier_local_attn_bwd(const ug_plan* plan, const void* q_hr, const void* k_
                            void* dk_hr, void* dv_hr, void* dq_lr, void* dk_lr, void* dv_lr,
                            void* workspace, int64_t workspace_bytes, void* stream);
 
+/* ug_hier_local_attn_bwd with the high-res v, o, dO read and dv written in
+ * raster order (q, k, dq, dk stay window-first; the global tensors as
+ * before), so that the layer's backward needs no permutes of v, o and dO and
+ * no unpermute of dv.  As ug_hier_local_attn_fwd_vo_raster, it needs every
+ * 128-row tile to be whole rows of one window: win_w dividing 128 and 128
+ * dividing win_h * win_w (UG_ERR_UNSUPPORTED otherwise).  Results equal the
+ * window-first call's, permuted, bit for bit.  ug_layer_bwd uses it where it
+ * applies. */
+int ug_hier_local_attn_bwd_vo_raster(const ug_plan* plan, const void* q_hr, const void* k_hr,
+                                     const void* v_hr_raster, const void* q_lr,
+                                     const void* k_lr, const void* v_lr,
+                                     const void* o_hr_raster, const void* o_lr,
+                                     const void* do_hr_raster, const void* do_lr,
+                                     const float* lse, void* dq_hr, void* dk_hr,
+                                     void* dv_hr_raster, void* dq_lr, void* dk_lr, void* dv_lr,
+                                     void* workspace, int64_t workspace_bytes, void* stream);
+
 /* Device scratch of ug_layer_bwd. */
 int64_t ug_layer_bwd_workspace_bytes(const ug_plan* plan);
 
@@ -336,8 +353,9 @@ int64_t ug_layer_bwd_workspace_bytes(const ug_plan* plan);
  * the layer's inputs q/k/v, its outputs o_hr (raster) / o_lr and lse, and
  * do_hr (raster) / do_lr, writes dq/dk/dv (same layouts as q/k/v; dq, dk
  * are gradients w.r.t. the unrotated q, k).  Recomputes the window-first,
- * rotated operands, runs ug_hier_local_attn_bwd, then the inverse
- * permutation with the transposed RoPE.  workspace: at least
+ * rotated operands, runs ug_hier_local_attn_bwd (or its raster variant where
+ * that applies: then v, o, dO are read and dv written in raster order
+ * directly), then the inverse permutation with the transposed RoPE.  workspace: at least
  * ug_layer_bwd_workspace_bytes, 256-byte aligned, disjoint from every
  * argument. */
 int ug_layer_bwd(const ug_plan* plan, const void* q_hr, const void* k_hr, const void* v_hr,

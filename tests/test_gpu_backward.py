@@ -196,6 +196,42 @@ def test_layer_backward_every_element(name):
     check(got[2], ref[2], bv, f"{name} layer dv")
 
 
+@pytest.mark.parametrize("name", SMALL + ["2K", "4K-CFG"])
+def test_attention_backward_raster_equals_permuted_path(name):
+    """ug_hier_local_attn_bwd_vo_raster (v, o, dO read and dv written in
+    raster order) gives bit for bit the window-first backward's gradients,
+    with dv unpermuted; geometries whose 128-row tiles are not whole window
+    rows are refused."""
+    wl = workloads.get(name)
+    p = plan(wl)
+    x = inputs(wl, 830)
+    d = {k: v.to(DEV) for k, v in x.items()}
+    has_lr = wl.n_lr > 0
+    g = lambda n: d[n] if has_lr else None
+    T = wl.win_h * wl.win_w
+    supported = 128 % wl.win_w == 0 and T % 128 == 0
+    o_hr, o_lr, lse = ug.hier_local_attn_fwd(p, d["q_hr"], d["k_hr"], d["v_hr"], g("q_lr"),
+                                             g("k_lr"), g("v_lr"))
+    ref = ug.hier_local_attn_bwd(p, d["q_hr"], d["k_hr"], d["v_hr"], g("q_lr"), g("k_lr"),
+                                 g("v_lr"), o_hr, o_lr, d["do_hr"], g("do_lr"), lse)
+    v_r, o_r, do_r = (ug.unpermute(p, t) for t in (d["v_hr"], o_hr, d["do_hr"]))
+    like = lambda t: torch.empty_like(t) if t is not None else None
+    outs = [like(t) for t in (d["q_hr"], d["k_hr"], d["v_hr"], g("q_lr"), g("k_lr"), g("v_lr"))]
+    ws = torch.empty(p.attn_bwd_workspace_bytes(), dtype=torch.uint8, device=DEV)
+    st = p.hier_local_attn_bwd_vo_raster(d["q_hr"], d["k_hr"], v_r, g("q_lr"), g("k_lr"),
+                                         g("v_lr"), o_r, o_lr, do_r, g("do_lr"), lse, *outs, ws)
+    if not supported:
+        assert st == ug.UG_ERR_UNSUPPORTED
+        return
+    assert st == ug.UG_OK, ug.status_string(st)
+    torch.cuda.synchronize()
+    assert p.check_error() == ug.UG_OK
+    assert torch.equal(outs[0], ref[0]) and torch.equal(outs[1], ref[1])
+    assert torch.equal(outs[2], ug.unpermute(p, ref[2]))
+    for a, b in zip(outs[3:], ref[3:]):
+        assert (a is None and b is None) or torch.equal(a, b)
+
+
 def test_backward_error_statuses():
     wl = workloads.get("tiny")
     p = plan(wl)
