@@ -52,12 +52,11 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on a barrier phase.  Gives up when the CTA's abort flag is up
-// (unless ignore_abort) or after timeout_ns; on a timeout it records the
-// status and raises the abort flag.  Returns true when the phase completed.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
-                                       int* err, int64_t timeout_ns, bool ignore_abort) {
-  if (mbar_test(bar, parity)) return true;
+// The polling loop of mbar_wait, out of line: reached only when the phase is
+// not complete at the first test.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+                                            volatile uint32_t* abort, int* err,
+                                            int64_t timeout_ns, bool ignore_abort) {
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
@@ -70,6 +69,18 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile u
       }
     }
   }
+}
+
+// Bounded wait on a barrier phase.  Gives up when the CTA's abort flag is up
+// (unless ignore_abort) or after timeout_ns; on a timeout it records the
+// status and raises the abort flag.  Returns true when the phase completed.
+// The first test is inline: a call costs the single-thread issuing roles
+// hundreds of cycles (measured), most often for a phase that is already
+// complete.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                          int* err, int64_t timeout_ns, bool ignore_abort) {
+  if (mbar_test(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort, err, timeout_ns, ignore_abort);
 }
 
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int32_t c0,
