@@ -25,7 +25,7 @@ namespace ug {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kRows = 4;  // output rows per thread
+constexpr int kRows = 8;  // output rows per thread
 
 struct WarmArgs {
   const float* x_lr;
