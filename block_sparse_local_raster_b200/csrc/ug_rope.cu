@@ -189,6 +189,12 @@ __global__ void __launch_bounds__(kThreads, 3) rope_rows_kernel(const RopeArgs a
     uint4* __restrict__ ys = a.y + dst * a.row_chunks;
     const AxisRow rr = axis_row(a.tables, a.row, pr, a.my);
     const AxisRow cc = axis_row(a.tables, a.col, pc, a.mx);
+    // A lane meets chunks lane, lane + 32, ...: when the head's chunk count
+    // divides 32 they all sit at the same place in their head, so the lane's
+    // angles are loaded once per row.
+    constexpr bool kFixed = HEAD_CHUNKS != 0 && 32 % (HEAD_CHUNKS ? HEAD_CHUNKS : 1) == 0;
+    rope_math::Angles4 fixed;
+    if (kFixed) fixed = chunk_angles(lane % hc, a.ay_chunks, rr, cc);
     for (int32_t c0 = lane; c0 < a.row_chunks; c0 += 32 * kUnroll) {
       uint4 v[kUnroll];
 #pragma unroll
@@ -200,7 +206,8 @@ __global__ void __launch_bounds__(kThreads, 3) rope_rows_kernel(const RopeArgs a
       for (int u = 0; u < kUnroll; ++u) {
         const int32_t c = c0 + 32 * u;
         if (c < a.row_chunks)
-          ys[c] = rotate_chunk<kTranspose>(v[u], chunk_angles(c % hc, a.ay_chunks, rr, cc));
+          ys[c] = rotate_chunk<kTranspose>(
+              v[u], kFixed ? fixed : chunk_angles(c % hc, a.ay_chunks, rr, cc));
       }
     }
   }

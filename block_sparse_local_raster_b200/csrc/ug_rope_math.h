@@ -32,9 +32,7 @@
 
 #include <cstdint>
 #include <cstring>
-#if !defined(__CUDACC__)
 #include <cmath>
-#endif
 
 #if defined(__CUDACC__)
 #define UG_RM_FN __host__ __device__ __forceinline__
@@ -100,12 +98,9 @@ UG_RM_FN uint32_t lower_bound(const uint32_t w[4]) {
   return (uint32_t)(lb > 0x21800000 ? lb : 0x21800000);  // 2^-60
 }
 
-// y is decided: |y| >= lb (bit patterns) and y at least 4 ulps from the bf16
-// midpoint of its binade (low 16 bits outside [0x7FFD, 0x8004]).
-UG_RM_FN bool decided(float y, uint32_t lb) {
-  const uint32_t b = as_u(y);
-  return (b & 0x7FFFFFFFu) >= lb && ((b + 3u) & 0xFFF8u) != 0x8000u;
-}
+// y at least 4 ulps from the bf16 midpoint of its binade (low 16 bits
+// outside [0x7FFD, 0x8004]).
+UG_RM_FN bool clear_of_midpoint(float y) { return ((as_u(y) + 3u) & 0xFFF8u) != 0x8000u; }
 
 // The cos/sin of a chunk's 4 pairs, split.
 struct Angles4 {
@@ -166,12 +161,17 @@ UG_RM_FN bool chunk_fast(const uint32_t w[4], const Angles4& t, uint32_t out[4])
     y1[k] = h1 + l1;
   }
 #endif
+  // every |y| >= lb (one comparison of the chunk's smallest |y|: no output
+  // of a chunk that passed lower_bound is infinite or NaN), and every y
+  // clear of its midpoint
+  float amin = std::fabs(y0[0]);
   bool ok = true;
   for (int k = 0; k < 4; ++k) {
-    ok = ok & decided(y0[k], lb) & decided(y1[k], lb);
+    amin = std::fmin(amin, std::fmin(std::fabs(y0[k]), std::fabs(y1[k])));
+    ok = ok & clear_of_midpoint(y0[k]) & clear_of_midpoint(y1[k]);
     out[k] = pack_bf16_rn(y0[k], y1[k]);
   }
-  return ok;
+  return ok & (as_u(amin) >= lb);
 }
 
 }  // namespace rope_math
