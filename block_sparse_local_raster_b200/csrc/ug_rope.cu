@@ -36,7 +36,7 @@ namespace ug {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;  // 16-byte chunks in flight per thread
+constexpr int kUnroll = 6;  // 16-byte chunks in flight per thread (4: 153 us, 6: 149 us per 4K tensor)
 
 // fp64 -> fp32 rounded to odd: truncate, then set the last bit if anything
 // was dropped.  For results in fp32's normal range the dropped part is the
