@@ -31,6 +31,9 @@
 // the tensor pipe executes in issue order, so S_t(j+1) overwrites P_t(j) only
 // after O_t += P_t(j) V_j has read it, and the commit that signals S_t(j+1)
 // also covers that product (the softmax never waits for O separately).
+// P_t is handed over in two halves (keys 0-63, then 64-127), so the first
+// half of O_t += P_t V_j runs while the softmax computes the second; each
+// softmax warp arrives once per half, after its own stores are complete.
 // Online softmax in the log2 domain with lazy rescaling: the running
 // reference max moves (and O, l are rescaled) only when a block's max exceeds
 // it by more than 8 (a factor 256), so probabilities stay <= 256 and O is
@@ -66,8 +69,9 @@ struct Layout {
   static constexpr int kQ = 0;
   static constexpr int kKV = kQ + kTilesPerCta * kTileBytes;
   static constexpr int kBar = kKV + kStages * kTileBytes;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 3 * kTilesPerCta + 1;
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain,
+  // p_half[2]
+  static constexpr int kNumBars = 1 + 2 * kStages + 4 * kTilesPerCta + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base (u32), abort flag (u32)
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
@@ -122,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto p_full = [&](int t) { return bar0 + 8u * (1 + 2 * kStages + 2 + t); };
   auto o_done = [&](int t) { return bar0 + 8u * (1 + 2 * kStages + 4 + t); };
   const uint32_t drain = bar0 + 8u * (1 + 2 * kStages + 6);
+  auto p_half = [&](int t) { return bar0 + 8u * (1 + 2 * kStages + 7 + t); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
   volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + Lay::kMisc + 4);
   int* const err = P.err;
@@ -156,7 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < kTilesPerCta; ++t) {
       mbar_init(s_full(t), 1);
-      mbar_init(p_full(t), kRowsPerTile);
+      mbar_init(p_half(t), 4);  // one arrive per softmax warp of the tile
+      mbar_init(p_full(t), 4);
       mbar_init(o_done(t), 1);
     }
     mbar_init(drain, 1);
@@ -262,12 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                    kk > 0);
         }
       };
-      // O_t += P_t V: P_t (bf16, 128 x 128) sits in the first 64 columns of
-      // S_t, 16 keys per 8 columns; V (keys x D, D contiguous) is MN-major.
-      auto issue_pv = [&](int t, int slot, bool acc) {
+      // O_t += P_t V over keys [16 kk0, 16 kk1): P_t (bf16, 128 x 128) sits in
+      // the first 64 columns of S_t, 16 keys per 8 columns; V (keys x D, D
+      // contiguous) is MN-major.
+      auto issue_pv = [&](int t, int slot, bool acc, int kk0, int kk1) {
         const uint32_t va = sbase + Lay::kKV + slot * Lay::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kKeysPerBlock / 16; ++kk)
+        for (int kk = kk0; kk < kk1; ++kk)
           mma_bf16_tmem_a(tO[t], tS[t] + kk * 8, smem_desc(va + kk * 16 * 128, kKeysPerBlock * 128, 1024),
                           kIdO, (acc || kk > 0) ? 1u : 0u);
       };
@@ -286,9 +293,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sv = itv % kStages, sk = itk % kStages;
         const bool more = j + 1 < nblk;
         if (!(ok = wait1(kv_full(sv), (uint32_t)(itv / kStages) & 1u))) break;
+        if (!(ok = wait1(p_half(0), (uint32_t)j & 1u))) break;
+        fence_after();
+        issue_pv(0, sv, j > 0, 0, kKeysPerBlock / 32);
         if (!(ok = wait1(p_full(0), (uint32_t)j & 1u))) break;
         fence_after();
-        issue_pv(0, sv, j > 0);
+        issue_pv(0, sv, true, kKeysPerBlock / 32, kKeysPerBlock / 16);
         if (!more) mma_commit(o_done(0));
         if (more) {
           if (!(ok = wait1(kv_full(sk), (uint32_t)(itk / kStages) & 1u))) break;
@@ -296,9 +306,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_s(0, sk);
           mma_commit(s_full(0));
         }
+        if (!(ok = wait1(p_half(1), (uint32_t)j & 1u))) break;
+        fence_after();
+        issue_pv(1, sv, j > 0, 0, kKeysPerBlock / 32);
         if (!(ok = wait1(p_full(1), (uint32_t)j & 1u))) break;
         fence_after();
-        issue_pv(1, sv, j > 0);
+        issue_pv(1, sv, true, kKeysPerBlock / 32, kKeysPerBlock / 16);
         if (!more) mma_commit(o_done(1));
         mma_commit(kv_empty(sv));
         if (more) {
@@ -321,6 +334,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tok = qt.q0 + t * kRowsPerTile + row;  // query token in its tensor
     const int q_w = tok / P.T;
     const int q_wy = q_w / P.nwx, q_wx = q_w - (q_w / P.nwx) * P.nwx;
+    // This warp's probability stores complete and ordered before the MMA
+    // warp's reads: wait for them, fence, then one arrive for the warp.
+    auto hand_over = [&](uint32_t bar) {
+      tmem_st_wait();
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
     float m_ref = kNegInf;  // reference max (log2 units) of the O/l accumulators
     float l = 0.0f;
     bool ok = true;
@@ -405,12 +426,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[i / 2] = pack_bf16(pp.x, pp.y);
         }
         tmem_st8u(tS + 8 * h, pk);
+        if (h == kKeysPerBlock / 32 - 1) hand_over(p_half(t));  // keys 0-63 stored
       }
       const float2 a4 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
       l = l * alpha + (a4.x + a4.y);
-      tmem_st_wait();
-      fence_before();
-      mbar_arrive(p_full(t));
+      hand_over(p_full(t));
     }
     // ------------------------------------------------------------ epilogue
     if (ok) ok = wait_warp(o_done(t), 0);
