@@ -240,6 +240,9 @@ WARM_START: Dict[str, WarmStart] = {
     "odd": WarmStart("odd", 2, 3, 13, 7, 3, sharpen=1.25, t=0.3),
     "s1": WarmStart("s1", 1, 2, 9, 20, 1),
     "wide": WarmStart("wide", 1, 1, 3, 70, 4, sharpen=0.0, t=0.0),
+    # factor 4 with every border case: odd sizes, a one-pixel-wide plane
+    "s4_edges": WarmStart("s4_edges", 2, 3, 5, 9, 4, sharpen=0.8, t=0.45),
+    "s4_thin": WarmStart("s4_thin", 1, 2, 1, 1, 4, sharpen=0.5, t=0.6),
 }
 
 
