@@ -98,7 +98,7 @@ EXTRA_CONFIGS: Dict[str, Workload] = {
 
 # Small geometries for element-by-element parity: several tiles, ragged tails,
 # non-square grids, windows that do not divide the 128-token tile, radius 0/2,
-# no low-res set, one window covering the whole grid.
+# no low-res set, one window covering the whole grid, 1024-token windows.
 TEST_GEOMETRIES: Dict[str, Workload] = {
     "multi_tile": _wl("multi_tile", 2, (64, 48), (16, 16), (12, 10), 3, 128, (64, 64)),
     "win12_d64": _wl("win12_d64", 1, (48, 36), (12, 12), (7, 5), 2, 64, (32, 32)),
@@ -113,6 +113,9 @@ TEST_GEOMETRIES: Dict[str, Workload] = {
     "text77": _wl("text77", 1, (48, 32), (16, 16), (6, 4), 2, 128, (64, 64), text_len=77),
     "text_only": _wl("text_only", 1, (32, 24), (8, 8), (0, 0), 2, 64, (32, 32),
                      text_len=130),
+    # the 1024-token windows of 4K-CFG (8 key blocks per window, raster v/o
+    # eligible) on a 3 x 2 window grid, where corner windows do not see the far row
+    "win32": _wl("win32", 1, (96, 64), (32, 32), (24, 16), 2, 128, (64, 64)),
 }
 
 

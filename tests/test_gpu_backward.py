@@ -125,6 +125,43 @@ def test_attention_backward_sampled_full_size(name):
     assert bool((tot(dk_hr, dk_lr).abs() <= 2 * U * mag(dk_hr, dk_lr) + 1e-3).all())
 
 
+def test_attention_backward_8K_sampled_rows():
+    """The 8K layer (262144 high-res tokens, 16384 global ones): dQ of
+    sampled query rows for two heads against the oracle under the derived
+    bounds, and the gradient-sum identities for every head and key.  Inputs
+    are drawn on the device with the same distributions (the CPU draw of 8K
+    takes minutes); the oracle reads the two heads back."""
+    wl = workloads.get("8K")
+    g = ogeom(wl)
+    p = plan(wl)
+    d = workloads.make_inputs_on_device(wl, 840, DEV)
+    gen = torch.Generator(device=DEV).manual_seed(841)
+    for name, n in (("do_hr", wl.n_hr), ("do_lr", wl.n_lr)):
+        d[name] = torch.randn((wl.batch, n, wl.heads, wl.head_dim), generator=gen,
+                              device=DEV).to(torch.bfloat16)
+    grads = forward_backward(p, wl, d)
+    heads = [0, 23]
+    rows = np.concatenate([sample_hr_tokens(g, O.HR_WINDOW_FIRST, 9, n_interior=2, per_window=2),
+                           g.N + sample_lr_tokens(g, 9, n=4)])
+    none = np.zeros(0, dtype=np.int64)
+    xb = {k: bits(v[:, :, heads]) for k, v in d.items()}
+    g1 = O.Geometry.from_dict(dict(wl.geom_dict(), heads=len(heads)))
+    ref = O.attention_backward(xb["q_hr"], xb["k_hr"], xb["v_hr"], xb["q_lr"], xb["k_lr"],
+                               xb["v_lr"], xb["do_hr"], xb["do_lr"], g1, O.HR_WINDOW_FIRST,
+                               rows=rows, keys=none)
+    bnd = bwd_error_bounds(g1, O.HR_WINDOW_FIRST,
+                           *(joint_f64(d, n, heads) for n in ("q", "k", "v", "do")),
+                           rows=rows, keys=none)
+    gq, _, _ = joint_grads(grads, wl, heads)
+    check(gq[:, rows], ref[0], bnd[0], "8K dq")
+    tot = lambda a, b_: a.double().sum(1) + b_.double().sum(1)
+    mag = lambda a, b_: a.double().abs().sum(1) + b_.double().abs().sum(1)
+    dk_hr, dv_hr, dk_lr, dv_lr = grads[1], grads[2], grads[4], grads[5]
+    do_sum = tot(d["do_hr"], d["do_lr"])
+    assert bool(((tot(dv_hr, dv_lr) - do_sum).abs() <= U * mag(dv_hr, dv_lr) + 1e-3).all())
+    assert bool((tot(dk_hr, dk_lr).abs() <= 2 * U * mag(dk_hr, dk_lr) + 1e-3).all())
+
+
 SETS = [(ug.UG_HR_WINDOW_FIRST, O.HR_WINDOW_FIRST), (ug.UG_HR_RASTER, O.HR_RASTER),
         (ug.UG_LR, O.LOWRES)]
 
