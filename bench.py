@@ -436,8 +436,11 @@ def time_steps(step, steps, warmup, dev, stream, rank, local, per_step_flush_byt
     step(ev) records ev[0] / ev[1] around the kernel it wants timed alone.
     When the inputs fit in L2 (per_step_flush_bytes > 0) a buffer of that
     size is written between steps and each step is timed by its own events,
-    so the flush is outside the time.  Returns (seconds per step, kernel
-    seconds per launch, clock record), max over ranks."""
+    so the flush is outside the time; otherwise an event between steps
+    splits the region into steps without adding to it.  Returns (seconds per
+    step, kernel seconds per launch, clock record), max over ranks, and this
+    rank's per-step distribution (median, p10, p90 of the step and of the
+    timed kernel, ms)."""
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -446,6 +449,7 @@ def time_steps(step, steps, warmup, dev, stream, rank, local, per_step_flush_byt
     mk = lambda: torch.cuda.Event(enable_timing=True)
     kev = [(mk(), mk()) for _ in range(steps)]
     sev = [(mk(), mk()) for _ in range(steps)] if flush is not None else None
+    bev = [mk() for _ in range(steps + 1)] if flush is None else None
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
@@ -458,9 +462,13 @@ def time_steps(step, steps, warmup, dev, stream, rank, local, per_step_flush_byt
         if flush is not None:
             flush.fill_(i & 0xFF)
             sev[i][0].record(stream)
+        else:
+            bev[i].record(stream)
         step(kev[i])
         if flush is not None:
             sev[i][1].record(stream)
+    if bev is not None:
+        bev[steps].record(stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -470,7 +478,13 @@ def time_steps(step, steps, warmup, dev, stream, rank, local, per_step_flush_byt
     else:
         sec = t0.elapsed_time(t1) / 1e3 / steps
     ksec = sum(a.elapsed_time(b) for a, b in kev) / 1e3 / steps
-    return reduce_max(sec, dev), reduce_max(ksec, dev), clk
+    per = ([a.elapsed_time(b) for a, b in sev] if sev is not None else
+           [bev[i].elapsed_time(bev[i + 1]) for i in range(steps)])
+    kper = [a.elapsed_time(b) for a, b in kev]
+    pct = lambda v: {"median": float(np.median(v)), "p10": float(np.percentile(v, 10)),
+                     "p90": float(np.percentile(v, 90))}
+    dist = {"step_ms": pct(per), "kernel_ms": pct(kper)}
+    return reduce_max(sec, dev), reduce_max(ksec, dev), clk, dist
 
 
 def layer_record(args, wl, d, dev, stream, rank, local, steps=None, warmup=None):
@@ -479,7 +493,7 @@ def layer_record(args, wl, d, dev, stream, rank, local, steps=None, warmup=None)
     steps = steps or args.steps
     warmup = warmup if warmup is not None else args.warmup
     flush = 0 if r.hr_bytes > L2_BYTES else 2 * L2_BYTES
-    sec, attn, clk = time_steps(r.step, steps, warmup, dev, stream, rank, local, flush)
+    sec, attn, clk, dist = time_steps(r.step, steps, warmup, dev, stream, rank, local, flush)
     _chk(r.plan.check_error(), f"{wl.name} timed steps")
     ach = r.flops / attn / 1e12
     rec = {
@@ -494,6 +508,7 @@ def layer_record(args, wl, d, dev, stream, rank, local, steps=None, warmup=None)
         "roofline": tensor_roofline(ach, attn * steps, clk,
                                     attn_traffic_bytes(wl.name)),
         "clocks": clk,
+        "per_step_ms": dist,
     }
     return r, rec
 
@@ -637,6 +652,7 @@ def run_ug(args, wl, world, rank, local):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": LayerRunner.launches_of(wl) * args.steps,
             "clocks": rec["clocks"],
+            "per_step_ms": rec["per_step_ms"],
             "per_config": per_config,
         }
         if bwd is not None:
@@ -651,6 +667,10 @@ def run_ug(args, wl, world, rank, local):
                 "nproc": cpu_cores(), "kind": "oracle",
                 "sample": (f"{len(arm.rows)} query rows x {wl.heads} heads of the {wl.name} "
                            f"layer (RoPE of every key included), fp64 numpy, {cdt:.1f} s"),
+                # rows are independent: the whole layer's useful FLOPs at the
+                # sample's rate (an upper estimate: the sample's RoPE of every
+                # key is a fixed cost that the extrapolation scales too)
+                "extrapolated_ms_per_layer": flops / (arm.flops / cdt) * 1e3,
             }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -731,7 +751,7 @@ def backward_record(args, wl, d, fwd, dev, stream, rank, local, steps=None):
     br = BackwardRunner(wl, d, fwd.plan, fwd.o_hr, fwd.o_lr, fwd.lse, dev)
     steps = steps or args.steps
     flush = 0 if fwd.hr_bytes > L2_BYTES else 2 * L2_BYTES
-    sec, attn, clk = time_steps(br.step, steps, max(3, min(args.warmup, 5)), dev, stream, rank,
+    sec, attn, clk, dist = time_steps(br.step, steps, max(3, min(args.warmup, 5)), dev, stream, rank,
                                 local, flush)
     _chk(fwd.plan.check_error(), "backward timed steps")
     ach = br.flops / attn / 1e12
@@ -744,6 +764,7 @@ def backward_record(args, wl, d, fwd, dev, stream, rank, local, steps=None):
         "roofline": tensor_roofline(ach, attn * steps, clk,
                                     note="7 products executed per visible pair, 5 counted"),
         "clocks": clk,
+        "per_step_ms": dist,
     }
 
 
@@ -765,7 +786,7 @@ def run_backward(args, wl, world, rank, local):
     fwd.step()
     br = BackwardRunner(wl, d, fwd.plan, fwd.o_hr, fwd.o_lr, fwd.lse, dev)
     flush = 0 if fwd.hr_bytes > L2_BYTES else 2 * L2_BYTES
-    sec, attn, clk = time_steps(br.step, args.steps, args.warmup, dev, stream, rank, local, flush)
+    sec, attn, clk, dist = time_steps(br.step, args.steps, args.warmup, dev, stream, rank, local, flush)
     plan, o_hr, o_lr, lse = fwd.plan, fwd.o_hr, fwd.o_lr, fwd.lse
     _chk(plan.check_error(), "timed steps")
     # end to end: inputs (q, k, v, o, lse, do) from pinned host memory, the
@@ -808,7 +829,7 @@ def run_backward(args, wl, world, rank, local):
                               if not flush else
                               "inputs smaller than L2 (%.0f MB per high-res tensor), flushed "
                               "between steps") % (d["q_hr"].numel() * 2 / 1e6)},
-            "attn_bwd_ms": attn * 1e3, "attn_bwd_tflops": ach,
+            "attn_bwd_ms": attn * 1e3, "attn_bwd_tflops": ach, "per_step_ms": dist,
             "roofline": tensor_roofline(ach, attn * args.steps, clk,
                                         note="7 products executed per visible pair, 5 counted"),
             "e2e": {"value": aggregate(flops, world, e2e_sec) / 1e12, "unit": "TFLOP/s",
