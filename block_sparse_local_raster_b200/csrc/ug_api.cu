@@ -629,6 +629,12 @@ int ug_warm_start(const ug_warm_start_params* q, const float* x_lr, const float*
   return launch_warm_start(q, x_lr, noise, out, as_stream(s));
 }
 
+int ug_warm_start_stencil_weights(float sharpen, float t, float* weights) {
+  if (!weights || !std::isfinite(sharpen) || !(t >= 0.0f && t <= 1.0f)) return UG_ERR_INVALID_ARG;
+  warm_start_stencil_weights(sharpen, t, weights);
+  return UG_OK;
+}
+
 int ug_check_error(const ug_plan* p, void* s) {
   if (!p) return UG_ERR_INVALID_ARG;
   if (const int st = check_device(p)) return st;

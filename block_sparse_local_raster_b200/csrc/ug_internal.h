@@ -120,6 +120,8 @@ int launch_attention_bwd(const ug_plan* p, const void* q_hr, const void* k_hr, c
                          void* dv_lr, float* delta, bool vo_raster, cudaStream_t s);
 int launch_warm_start(const ug_warm_start_params* p, const float* x_lr, const float* noise,
                       float* out, cudaStream_t s);
+// The factor-4 warm start's weights, [py][px][3 r + c] (host, fp64 -> fp32).
+void warm_start_stencil_weights(double amount, double t, float* wt);
 int launch_attention(const ug_plan* p, const void* q_hr, const void* k_hr, const void* v_hr,
                      const void* q_lr, const void* k_lr, const void* v_lr, void* o_hr,
                      void* o_lr, float* lse, bool vo_raster, cudaStream_t s);

@@ -257,8 +257,11 @@ __global__ void __launch_bounds__(kStencilThreads) warm_start_stencil_kernel(con
   }
 }
 
-// W of the stencil for factor s = kStencilS, in fp64, rounded once to fp32.
-void stencil_weights(double amount, double t, float wt[kStencilS][kStencilS][9]) {
+}  // namespace
+
+// W of the stencil for factor s = kStencilS, in fp64, rounded once to fp32,
+// as [py][px][3 r + c].
+void warm_start_stencil_weights(double amount, double t, float* wt) {
   constexpr int S = kStencilS;
   // bilinear weights over source rows (Y-1, Y, Y+1) of the high-res row
   // S*Y + p + a, a in {-1, 0, 1}: source coordinate Y + q, q = (p + a +
@@ -281,11 +284,10 @@ void stencil_weights(double amount, double t, float wt[kStencilS][kStencilS][9])
     for (int px = 0; px < S; ++px)
       for (int r = 0; r < 3; ++r)
         for (int c = 0; c < 3; ++c)
-          wt[py][px][3 * r + c] = (float)((1.0 - t) * ((1.0 + amount) * e[py][r] * e[px][c] -
-                                                       amount * f[py][r] * f[px][c]));
+          wt[(py * S + px) * 9 + 3 * r + c] =
+              (float)((1.0 - t) * ((1.0 + amount) * e[py][r] * e[px][c] -
+                                   amount * f[py][r] * f[px][c]));
 }
-
-}  // namespace
 
 int launch_warm_start(const ug_warm_start_params* p, const float* x_lr, const float* noise,
                       float* out, cudaStream_t st) {
@@ -309,7 +311,7 @@ int launch_warm_start(const ug_warm_start_params* p, const float* x_lr, const fl
     sa.w = p->lr_w;
     sa.n = (int64_t)p->batch * p->channels * p->lr_h * p->lr_w;
     sa.t = p->t;
-    stencil_weights(p->sharpen, p->t, sa.wt);
+    warm_start_stencil_weights(p->sharpen, p->t, &sa.wt[0][0][0]);
     const int64_t blocks = (sa.n + kStencilThreads - 1) / kStencilThreads;
     warm_start_stencil_kernel<<<(unsigned)blocks, kStencilThreads, 0, st>>>(sa);
     return cudaGetLastError() == cudaSuccess ? UG_OK : UG_ERR_CUDA;

@@ -41,7 +41,7 @@ EXPORTS = (
     "ug_permute_window_first", "ug_permute_rope_window_first", "ug_unpermute", "ug_rope_2d",
     "ug_hier_local_attn_fwd", "ug_hier_local_attn_fwd_vo_raster",
     "ug_layer_workspace_bytes", "ug_layer_fwd", "ug_layer_fwd_static_scratch",
-    "ug_plan_set_wait_timeout", "ug_check_error", "ug_warm_start",
+    "ug_plan_set_wait_timeout", "ug_check_error", "ug_warm_start", "ug_warm_start_stencil_weights",
     "ug_rope_2d_bwd", "ug_unpermute_rope_bwd", "ug_attn_bwd_workspace_bytes",
     "ug_hier_local_attn_bwd", "ug_hier_local_attn_bwd_vo_raster",
     "ug_layer_bwd_workspace_bytes", "ug_layer_bwd",
@@ -141,6 +141,8 @@ def _load(path: str) -> ctypes.CDLL:
         "ug_plan_set_wait_timeout": (I32, [P, I64]),
         "ug_check_error": (I32, [P, P]),
         "ug_warm_start": (I32, [ctypes.POINTER(ug_warm_start_params), P, P, P, P]),
+        "ug_warm_start_stencil_weights": (I32, [ctypes.c_float, ctypes.c_float,
+                                                ctypes.POINTER(ctypes.c_float)]),
         "ug_rope_2d_bwd": (I32, [P, P, P, I32, P]),
         "ug_unpermute_rope_bwd": (I32, [P, P, P, P]),
         "ug_attn_bwd_workspace_bytes": (I64, [P]),
@@ -441,6 +443,16 @@ def warm_start_raw(x_lr: torch.Tensor, noise: torch.Tensor, out: torch.Tensor, s
     prm = ug_warm_start_params(B, C, h, w, int(scale), float(sharpen), float(t))
     return lib().ug_warm_start(ctypes.byref(prm), _ptr(x_lr), _ptr(noise), _ptr(out),
                                _stream(stream))
+
+
+def warm_start_stencil_weights(sharpen: float, t: float):
+    """ug_warm_start_stencil_weights (host only): the factor-4 warm start's
+    weights as a [4, 4, 3, 3] numpy array ([py, px, r, c])."""
+    w = np.zeros(144, dtype=np.float32)
+    _check(lib().ug_warm_start_stencil_weights(
+        float(sharpen), float(t), w.ctypes.data_as(ctypes.POINTER(ctypes.c_float))),
+        "ug_warm_start_stencil_weights")
+    return w.reshape(4, 4, 3, 3)
 
 
 def warm_start(x_lr: torch.Tensor, noise: torch.Tensor, scale: int, sharpen: float, t: float,

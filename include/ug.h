@@ -397,6 +397,21 @@ typedef struct ug_warm_start_params {
 int ug_warm_start(const ug_warm_start_params* params, const float* x_lr, const float* noise,
                   float* out, void* stream);
 
+/* Host only (no GPU needed): the weights ug_warm_start applies for factor
+ * s = 4.  The map above is linear in x_lr, and output pixel (4Y + py,
+ * 4X + px) of a plane depends only on the 3 x 3 low-res neighbourhood of
+ * (Y, X):
+ *   out = sum_{r, c = 0..2} weights[(4 py + px) * 9 + 3 r + c]
+ *                           * x_lr[clamp(Y + r - 1)][clamp(X + c - 1)] + t * noise,
+ * indices clamped to the image (which also gives the blur's edge
+ * replication: the high-res rows and columns just outside the image sample
+ * only clamped source pixels, so they equal the border ones).  Writes the
+ * UG_WARM_START_STENCIL_WEIGHTS fp32 weights, computed in fp64 and rounded
+ * once; the caller owns the array.  UG_ERR_INVALID_ARG for a NULL pointer, a
+ * non-finite sharpen or t outside [0, 1]. */
+#define UG_WARM_START_STENCIL_WEIGHTS 144
+int ug_warm_start_stencil_weights(float sharpen, float t, float* weights);
+
 /* ---- errors ---------------------------------------------------------------- */
 
 /* Bound, in ns, on each device-side wait of this plan's attention kernel
