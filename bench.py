@@ -139,7 +139,11 @@ def _nvml_handle(device_index: int):
 class ClockSampler:
     """SM clock, power and clock-event reasons sampled during the timed
     region, read-only: NVML every 10 ms from a thread (nvidia-smi at 20 ms if
-    NVML is unavailable)."""
+    NVML is unavailable).  Each sample carries its host time; stop(t0, t1)
+    summarises the samples taken between t0 and t1 (the timed region), or,
+    when that window holds fewer than 3 (a region of a few tens of ms, or a
+    slow NVML), those of the region and the warm-up just before it, and says
+    which."""
 
     SMI = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
            "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -150,7 +154,7 @@ class ClockSampler:
     def __init__(self, device_index: int, period_s: float = 0.01):
         self.dev = device_index
         self.period = period_s
-        self.rows = []  # (sm_mhz, sm_max_mhz, power_w, reason bits)
+        self.rows = []  # (sm_mhz, sm_max_mhz, power_w, reason bits, host time)
         self.thread = None
         self.proc = None
         self.stop_flag = False
@@ -164,7 +168,7 @@ class ClockSampler:
                 sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
                 pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
                 rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.rows.append((float(sm), float(smax), pw, int(rs)))
+                self.rows.append((float(sm), float(smax), pw, int(rs), time.perf_counter()))
             except Exception:
                 pass
             time.sleep(self.period)
@@ -189,7 +193,7 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
         if self.thread is not None:
             self.stop_flag = True
             self.thread.join(timeout=5)
@@ -204,13 +208,23 @@ class ClockSampler:
                 r = line.split(", ")
                 try:
                     bits = sum(b for (_, b), v in zip(self.REASONS, r[5:9]) if v.strip() == "Active")
-                    self.rows.append((float(r[1]), float(r[2]), float(r[3]), bits))
+                    self.rows.append((float(r[1]), float(r[2]), float(r[3]), bits, None))
                 except (ValueError, IndexError):
                     continue
             os.unlink(self.out.name)
         else:
             return None
-        return self.summary(self.rows)
+        rows, window = self.rows, "whole sampling"
+        if t0 is not None and all(r[4] is not None for r in rows):
+            inside = [r for r in rows if t0 <= r[4] <= t1]
+            if len(inside) >= 3:
+                rows, window = inside, "timed region"
+            else:
+                rows, window = [r for r in rows if r[4] <= t1], "timed region and the warm-up before it"
+        out = self.summary(rows)
+        if out:
+            out["window"] = window
+        return out
 
     def summary(self, rows):
         if not rows:
@@ -441,6 +455,9 @@ def time_steps(step, steps, warmup, dev, stream, rank, local, per_step_flush_byt
     step, kernel seconds per launch, clock record), max over ranks, and this
     rank's per-step distribution (median, p10, p90 of the step and of the
     timed kernel, ms)."""
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -450,13 +467,10 @@ def time_steps(step, steps, warmup, dev, stream, rank, local, per_step_flush_byt
     kev = [(mk(), mk()) for _ in range(steps)]
     sev = [(mk(), mk()) for _ in range(steps)] if flush is not None else None
     bev = [mk() for _ in range(steps + 1)] if flush is None else None
-    clocks = ClockSampler(local) if rank == 0 else None
-    if clocks:
-        clocks.start()
-        time.sleep(0.05)
     barrier()
     torch.cuda.synchronize(dev)
     t0, t1 = mk(), mk()
+    h0 = time.perf_counter()
     t0.record(stream)
     for i in range(steps):
         if flush is not None:
@@ -471,8 +485,9 @@ def time_steps(step, steps, warmup, dev, stream, rank, local, per_step_flush_byt
         bev[steps].record(stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
+    h1 = time.perf_counter()
     barrier()
-    clk = clocks.stop() if clocks else None
+    clk = clocks.stop(h0, h1) if clocks else None
     if sev is not None:
         sec = sum(a.elapsed_time(b) for a, b in sev) / 1e3 / steps
     else:
@@ -505,7 +520,7 @@ def layer_record(args, wl, d, dev, stream, rank, local, steps=None, warmup=None)
               ("inputs smaller than L2 (%.0f MB per high-res tensor): a %d MB buffer is "
                "written between steps, outside each step's events" % (r.hr_bytes / 1e6,
                                                                        flush >> 20)),
-        "roofline": tensor_roofline(ach, attn * steps, clk,
+        "roofline": tensor_roofline(ach, sec * steps, clk,
                                     attn_traffic_bytes(wl.name)),
         "clocks": clk,
         "per_step_ms": dist,
@@ -761,7 +776,7 @@ def backward_record(args, wl, d, fwd, dev, stream, rank, local, steps=None):
         "layer_backward_tflops": br.flops / sec / 1e12, "attn_bwd_ms": attn * 1e3,
         "attn_bwd_tflops": ach, "useful_flop_per_backward": br.flops,
         "gpu_launches_per_step": br.launches,
-        "roofline": tensor_roofline(ach, attn * steps, clk,
+        "roofline": tensor_roofline(ach, sec * steps, clk,
                                     note="7 products executed per visible pair, 5 counted"),
         "clocks": clk,
         "per_step_ms": dist,
@@ -830,7 +845,7 @@ def run_backward(args, wl, world, rank, local):
                               "inputs smaller than L2 (%.0f MB per high-res tensor), flushed "
                               "between steps") % (d["q_hr"].numel() * 2 / 1e6)},
             "attn_bwd_ms": attn * 1e3, "attn_bwd_tflops": ach, "per_step_ms": dist,
-            "roofline": tensor_roofline(ach, attn * args.steps, clk,
+            "roofline": tensor_roofline(ach, sec * args.steps, clk,
                                         note="7 products executed per visible pair, 5 counted"),
             "e2e": {"value": aggregate(flops, world, e2e_sec) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": sum(v.numel() * v.element_size()
@@ -896,22 +911,23 @@ def run_warm_start(args, world, rank, local):
         if st != ug.UG_OK:
             raise ug.UgError(st, "ug_warm_start")
 
+    clocks = ClockSampler(local)
+    clocks.start()
     for i in range(args.warmup):
         launch(i)
     torch.cuda.synchronize(dev)
     barrier()
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)  # the sampler's first reading lands before the timed region
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
+    h0 = time.perf_counter()
     e0.record(stream)
     for i in range(args.steps):
         launch(i)
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    h1 = time.perf_counter()
     barrier()
-    clk = clocks.stop()
+    clk = clocks.stop(h0, h1)
     sec = reduce_max(e0.elapsed_time(e1) / 1e3 / args.steps, dev)
     # end to end: pinned host buffers in, result out, every step
     pin_lr, pin_noise = host["x_lr"].pin_memory(), host["noise"].pin_memory()
